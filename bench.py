@@ -1,0 +1,401 @@
+"""Benchmark of the MLA paged-KV decode hot path on B200.
+
+One step = the whole hot path over one batch: split-KV schedule
+(mla_get_metadata) + decode kernel + split-KV combine (mla_decode_fwd), all
+through the C ABI.  Inputs are resident in HBM before the timed region; L2 is
+flushed (256 MiB write) before every timed step and each step is timed with
+CUDA events on the launching stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
+replica of the workload (requests are independent, there is no data-path
+collective); the time is the max over ranks and `value` aggregates all ranks.
+`--impl reference` times the float64 CPU oracle on a bounded sample instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MLA decode TFLOPS & effective HBM GB/s on 1 B200 (frac of roofline)"
+DEFAULT_WORKLOAD = "uniform_bf16"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (what the method must move / compute)
+# ---------------------------------------------------------------------------
+
+def algorithmic_work(w: W.Workload, seqlens: np.ndarray):
+    """Bytes and flops of one pass, counting valid tokens and visible pairs only.
+
+    bytes = sum_b L_b * T  (T = 1152 bf16 / 656 fp8 per token)
+          + |q| + |out| + |lse| + 4 * sum_b ceil(L_b / 64) (block-table reads) + 4 b (seqlens)
+    flops = 2 * (576 + 512) * h_q * sum over (request, query token) of visible keys
+    """
+    T = 1152 if w.fmt == "bf16" else 656
+    L = seqlens.astype(np.int64)
+    B = L.size
+    kv = int(L.sum()) * T
+    q = B * w.s_q * w.h_q * 576 * 2
+    out = B * w.s_q * w.h_q * 512 * 2
+    lse = B * w.s_q * w.h_q * 4
+    meta = 4 * int(((L + 63) // 64).sum()) + 4 * B
+    vis = 0
+    for i in range(w.s_q):
+        vis += int(np.clip(L - w.s_q + i + 1, 0, None).sum()) if w.causal else int(L.sum())
+    flops = 2 * (576 + 512) * w.h_q * vis
+    return dict(bytes=kv + q + out + lse + meta, kv_bytes=kv, flops=flops)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=FALLBACK_HBM_GBS, bf16_tflops=FALLBACK_BF16_TFLOPS,
+                bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+        self.gpu = gpu_index
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={CLOCK_QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = max((num(r[2]) for r in rows if num(r[2]) is not None), default=None)
+        loaded = [s for s in sm if smax and s >= 0.3 * smax] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle as a timed baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def oracle_rate(w: W.Workload, budget_s: float = 12.0, seed: int = 0):
+    """Time the float64 oracle on whole requests of the workload until `budget_s`.
+
+    Returns (GB/s of algorithmic bytes, sample description, cores used).
+    """
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    # whole requests of the workload, generated once on the CPU with its recipe
+    # and cycled until the time budget is spent
+    pool = []
+    for b in range(4):
+        one = W.Workload(w.name, 1, w.s_q, w.h_q, w.seqlen, fmt=w.fmt, causal=w.causal, seed=seed + b)
+        a = W.oracle_arrays(W.make_case(one, poison=False))
+        pool.append((a, algorithmic_work(one, a["cache_seqlens"])["bytes"]))
+    n_done, t_total, bytes_done = 0, 0.0, 0
+    while t_total < budget_s and n_done < 4096:
+        a, nbytes = pool[n_done % len(pool)]
+        t0 = time.perf_counter()
+        oracle.mla_decode(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
+                          a["softmax_scale"], a["causal"])
+        t_total += time.perf_counter() - t0
+        bytes_done += nbytes
+        n_done += 1
+    sample = f"{n_done} whole requests of {w.describe()} ({t_total:.1f} s of oracle time)"
+    return bytes_done / t_total / 1e9, sample, cores, t_total / max(n_done, 1)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    per_step = []
+    rate_bytes = 0
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        gbs, sample, cores, _ = oracle_rate(w, budget_s=budget, seed=1000 * i)
+        if i >= args.warmup:
+            per_step.append(gbs)
+    value = statistics.mean(per_step)
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.describe(), "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
+                       "seqlen": list(w.seqlen), "kv_format": w.fmt},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {sample}"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_cuda(args, world, rank, local):
+    import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    mla.load_library()
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    case = W.make_case(w, seed=w.seed + rank, device=dev, poison=False)
+    q, kv, bt, L = case["q"], case["kv_cache"], case["block_table"], case["cache_seqlens"]
+    B, s_q, h_q = w.batch, w.s_q, w.h_q
+    parts = args.parts or mla.mla_default_num_sm_parts(dev)
+    sched = torch.empty(mla.mla_metadata_size(B, parts) // 4, dtype=torch.int32, device=dev)
+    ns = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    ws = mla.alloc_workspace(B, s_q, h_q, parts, dev)
+    out = torch.empty((B, s_q, h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    seqlens_np = L.cpu().numpy()
+    work = algorithmic_work(w, seqlens_np)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
+        mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
+                           stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    status = mla.mla_last_device_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status {mla.STATUS.get(status, status)} during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index or 0) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
+            ev[i][1].record(stream)
+            mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
+                               stream=stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    meta_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    status = mla.mla_last_device_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status {mla.STATUS.get(status, status)} in the timed region")
+
+    # end to end through the public API: per step, H2D of the step's inputs
+    # (q, block table, sequence lengths) from pinned host memory, the decode,
+    # and D2H of its results (out, lse).  The paged KV cache is resident state.
+    q_h = q.cpu().pin_memory()
+    bt_h = bt.cpu().pin_memory()
+    L_h = L.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    q_d, bt_d, L_d = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(L)
+    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + L_h.numel() * 4
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q_d.copy_(q_h, non_blocking=True)
+        bt_d.copy_(bt_h, non_blocking=True)
+        L_d.copy_(L_h, non_blocking=True)
+        mla.mla_get_metadata(L_d, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
+        mla.mla_decode_fwd(q_d, kv, w.fmt, bt_d, L_d, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
+                           stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = max_over_ranks(sum(e2e_ms), world)
+
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    n = world
+    ms_per_step = total_ms / args.steps
+    value = n * work["bytes"] / (ms_per_step * 1e-3) / 1e9
+    tflops = n * work["flops"] / (ms_per_step * 1e-3) / 1e12
+    dec_avg = statistics.mean(dec_ms)
+    achieved = work["bytes"] / (dec_avg * 1e-3) / 1e9
+    compute_bound = work["flops"] / work["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if compute_bound:
+        ach_tf = work["flops"] / (dec_avg * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach_tf / peaks["bf16_tflops"], "traffic": None}
+    else:
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+    roof.update({"kernel": "decode (+ split-KV combine) via mla_decode_fwd", "peak_source": peaks["source"],
+                 "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
+                 "avg_ms": dec_avg})
+    traffic_file = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
+    if os.path.exists(traffic_file):
+        with open(traffic_file) as f:
+            roof["traffic"] = json.load(f).get("dram_bytes_per_launch")
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, sample, cores, _ = oracle_rate(w, budget_s=args.cpu_budget)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.describe(), "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
+                   "seqlen": list(w.seqlen), "kv_format": w.fmt, "causal": w.causal, "num_sm_parts": parts,
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replicas x{n} (independent request batches)"},
+        "tflops": tflops,
+        "metadata_ms": statistics.mean(meta_ms),
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": n * work["bytes"] / (e2e_total / args.steps * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_total / args.steps},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--parts", type=int, default=0, help="CTA pairs (default: SMs / 2)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_cuda(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

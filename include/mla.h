@@ -1,0 +1,143 @@
+/*
+ * mla.h — C ABI of the B200 (sm_100a) MLA paged-KV decoding library.
+ *
+ * Operation (FlashMLA, described on the pages as an "efficient MLA decoding
+ * kernel ... optimized for variable-length sequences", BF16, "Paged KV cache
+ * (block size 64)": DeepSeek launch tweet quoted on the 8bitnewsroom page;
+ * MLA's shared compressed latent KV with decoupled RoPE: Novita AI page,
+ * section "Was ist MLA?" and its MHA/MQA/GQA/MLA table):
+ *
+ *   For request b with L = cache_seqlens[b] cached tokens, query token i in
+ *   [0, s_q) and head h in [0, h_q):
+ *     K_j   = key of token j: 576 values (512 latent + 64 RoPE), read from
+ *             physical block block_table[b, j / 64], slot j % 64
+ *     V_j   = K_j[0:512]           (the value is the latent part of the key)
+ *     x_j   = softmax_scale * sum_{d<576} q[b,i,h,d] * K_j[d]
+ *     visible keys: j < L, and with causal != 0 also j <= L - s_q + i
+ *     lse[b,i,h]   = ln sum_j exp(x_j)                (natural log)
+ *     out[b,i,h,:] = sum_j exp(x_j - lse) * V_j       (bf16, RNE)
+ *   A row with no visible key gets out = 0 and lse = -inf.
+ *
+ * Cache formats:
+ *   MLA_KV_BF16     kv_cache is bf16 [num_blocks, 64, 576] (1152 B/token).
+ *   MLA_KV_FP8_656  kv_cache is uint8 [num_blocks, 64, 656] (656 B/token,
+ *                   the size on the menfem.com DeepSeek page, "Key
+ *                   Contributions"): bytes [0,512) E4M3 latent codes (OCP
+ *                   FP8 E4M3), bytes [512,528) four little-endian fp32 scales
+ *                   (scale g applies to latent dims [128g, 128g+128)), bytes
+ *                   [528,656) the 64 RoPE values in bf16.  The kernel forms
+ *                   code * scale in fp32 and rounds it to bf16 before the MMA.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps them after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it; nothing synchronises
+ *     except mla_last_device_status().
+ *   - Host-detectable argument errors return immediately (nothing enqueued).
+ *   - Errors the GPU detects (a block index outside [0, num_blocks), a wait
+ *     that exceeded its time limit) are recorded in a status word inside the
+ *     workspace; the first error recorded is kept until cleared.
+ *   - Supported shapes: d_qk 576, d_v 512, one latent KV head, 64-token
+ *     blocks, M = s_q * h_q rows per request with 1 <= M <= 128, bf16 q/out,
+ *     fp32 lse; q, kv_cache and out 16-byte aligned; batch <= 16384.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misalignment, non-finite scale */
+  MLA_ERR_UNSUPPORTED = 2,     /* shape outside the supported set, or no sm_100 device */
+  MLA_ERR_WORKSPACE = 3,       /* workspace or schedule buffer too small */
+  MLA_ERR_CUDA = 4,            /* a CUDA runtime/driver call or launch failed */
+  MLA_ERR_TIMEOUT = 5,         /* device: a bounded wait gave up (kernel returned early) */
+  MLA_ERR_BAD_BLOCK_INDEX = 6  /* device: block_table entry outside [0, num_blocks) */
+} mla_status_t;
+
+typedef enum { MLA_KV_BF16 = 0, MLA_KV_FP8_656 = 1 } mla_kv_format_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mla_status_string(mla_status_t status);
+
+/* Number of CTA pairs ("SM parts") the decode kernel should use on `device`:
+ * half the SM count (74 on a 148-SM B200).  Returns <= 0 if the device cannot
+ * be queried. */
+int mla_default_num_sm_parts(int device);
+
+/* Bytes of the int32 schedule buffer `sched` for mla_get_metadata. */
+size_t mla_metadata_size(int batch, int num_sm_parts);
+
+/*
+ * Split-KV schedule (the split-KV idea follows from "optimized for
+ * variable-length sequences" on the 8bitnewsroom page; the pages give no
+ * algorithm, this one is our own).  Every request costs ceil(L/64) pages
+ * plus a fixed per-request overhead; the concatenated cost line is cut into
+ * num_sm_parts equal pieces, so a request may be split across CTA pairs.
+ *
+ *   cache_seqlens  device int32 [batch], each >= 0
+ *   s_q, h_q       query tokens and heads per request (only validated here)
+ *   num_sm_parts   CTA pairs the decode launch will use (>= 1)
+ *   sched          device int32 buffer of mla_metadata_size() bytes (output)
+ *   num_splits     device int32 [batch + 1] (output): exclusive prefix sum of
+ *                  the number of splits per request; request b has
+ *                  num_splits[b+1] - num_splits[b] splits.
+ * The same `sched`/`num_splits` are valid for any decode call with the same
+ * cache_seqlens and num_sm_parts.  One tiny kernel, enqueued on `stream`.
+ */
+mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                              int num_sm_parts, int32_t* sched, int32_t* num_splits,
+                              void* stream);
+
+/* Bytes of workspace mla_decode_fwd needs: a status word plus fp32 partial
+ * outputs and partial lse for split requests.  Zero-fill it once after
+ * allocation (that clears the device status word). */
+size_t mla_workspace_size(int batch, int s_q, int h_q, int num_sm_parts);
+
+/*
+ * MLA decode over a paged cache (the hot path).
+ *
+ *   q              device bf16 [batch, s_q, h_q, 576], row-major
+ *   kv_cache       device, fmt-dependent (see above), [num_blocks, 64, ...]
+ *   fmt            MLA_KV_BF16 or MLA_KV_FP8_656
+ *   num_blocks     number of physical 64-token blocks in kv_cache (>= 1)
+ *   block_table    device int32 [batch, max_pages]; only the first
+ *                  ceil(L_b/64) entries of row b are read
+ *   max_pages      row stride of block_table (>= 1)
+ *   cache_seqlens  device int32 [batch]; L_b <= 64 * max_pages
+ *   softmax_scale  finite multiplier of the logits (576^-0.5 in the configs)
+ *   causal         non-zero: bottom-right causal mask among the s_q tokens
+ *   sched, num_splits  from mla_get_metadata with the same num_sm_parts
+ *   out            device bf16 [batch, s_q, h_q, 512] (output)
+ *   lse            device fp32 [batch, s_q, h_q] (output)
+ *   workspace      device buffer of >= mla_workspace_size() bytes
+ * Enqueues the decode kernel and, when some request is split, the split-KV
+ * combine kernel on `stream`.  Tail slots of a request's last page and blocks
+ * it does not reference may hold any bits (NaN/Inf included).
+ */
+mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt,
+                            int64_t num_blocks, const int32_t* block_table, int max_pages,
+                            const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                            float softmax_scale, int causal, const int32_t* sched,
+                            const int32_t* num_splits, int num_sm_parts, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the device-detected status recorded in
+ * `workspace` (MLA_OK if none) or MLA_ERR_CUDA if the stream reports an error. */
+mla_status_t mla_last_device_status(const void* workspace, void* stream);
+
+/* Enqueues a reset of the workspace status word to MLA_OK on `stream`. */
+mla_status_t mla_clear_device_status(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H_ */

@@ -1,0 +1,223 @@
+// C-ABI entry points (include/mla.h): argument validation, TMA descriptor
+// creation, workspace carving and kernel launches.  No allocation happens
+// here; every buffer belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+
+namespace mla {
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int parts, int32_t* sched, int32_t* num_splits,
+                            cudaStream_t stream);
+int metadata_max_batch();
+cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream);
+cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
+                               int num_parts, cudaStream_t stream);
+cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_tail, const DecodeParams& p,
+                              int num_parts, cudaStream_t stream);
+}  // namespace mla
+
+using namespace mla;
+
+namespace {
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// True if the current device is an sm_100 part (the only target built).
+bool device_supported() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+  return major == 10 && minor == 0;
+}
+
+// 2-D tiled map over a [rows, width] row-major cache view.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t width, uint64_t rows,
+              uint64_t row_bytes, uint32_t box_w, uint32_t box_h, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {width, rows};
+  cuuint64_t gstride[1] = {row_bytes};
+  cuuint32_t box[2] = {box_w, box_h};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+mla_status_t check_shape(int batch, int s_q, int h_q) {
+  if (batch < 1 || s_q < 1 || h_q < 1) return MLA_ERR_INVALID_ARG;
+  if (batch > metadata_max_batch()) return MLA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(s_q) * h_q > kRows) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+    case MLA_ERR_BAD_BLOCK_INDEX: return "MLA_ERR_BAD_BLOCK_INDEX";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+int mla_default_num_sm_parts(int device) {
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return -1;
+  return sms / 2;
+}
+
+size_t mla_metadata_size(int batch, int num_sm_parts) {
+  if (batch < 1 || num_sm_parts < 1) return 0;
+  return sched_ints(batch, num_sm_parts) * sizeof(int32_t);
+}
+
+mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int num_sm_parts,
+                              int32_t* sched, int32_t* num_splits, void* stream) {
+  if (!cache_seqlens || !sched || !num_splits) return MLA_ERR_INVALID_ARG;
+  if (!aligned(cache_seqlens, 4) || !aligned(sched, 16) || !aligned(num_splits, 4)) return MLA_ERR_INVALID_ARG;
+  if (num_sm_parts < 1 || num_sm_parts > 65535) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = check_shape(batch, s_q, h_q);
+  if (st != MLA_OK) return st;
+  cudaError_t e = launch_metadata(cache_seqlens, batch, num_sm_parts, sched, num_splits,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+size_t mla_workspace_size(int batch, int s_q, int h_q, int num_sm_parts) {
+  if (check_shape(batch, s_q, h_q) != MLA_OK || num_sm_parts < 1) return 0;
+  return ws_bytes(batch, num_sm_parts, s_q * h_q);
+}
+
+mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt, int64_t num_blocks,
+                            const int32_t* block_table, int max_pages, const int32_t* cache_seqlens, int batch,
+                            int s_q, int h_q, float softmax_scale, int causal, const int32_t* sched,
+                            const int32_t* num_splits, int num_sm_parts, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!q || !kv_cache || !block_table || !cache_seqlens || !sched || !num_splits || !out || !lse || !workspace)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv_cache, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+      !aligned(block_table, 4) || !aligned(cache_seqlens, 4) || !aligned(lse, 4) || !aligned(sched, 16) ||
+      !aligned(num_splits, 4))
+    return MLA_ERR_INVALID_ARG;
+  if (fmt != MLA_KV_BF16 && fmt != MLA_KV_FP8_656) return MLA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || num_blocks > (static_cast<int64_t>(1) << 31) / kPage) return MLA_ERR_INVALID_ARG;
+  if (max_pages < 1 || num_sm_parts < 1 || num_sm_parts > 65535) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = check_shape(batch, s_q, h_q);
+  if (st != MLA_OK) return st;
+  const int M = s_q * h_q;
+  if (workspace_bytes < ws_bytes(batch, num_sm_parts, M)) return MLA_ERR_WORKSPACE;
+  if (!device_supported()) return MLA_ERR_UNSUPPORTED;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.sched = sched;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.lse_part = reinterpret_cast<float*>(ws + ws_lse_offset());
+  p.o_part = reinterpret_cast<float*>(ws + ws_o_offset(batch, num_sm_parts, M));
+  p.status = reinterpret_cast<int*>(ws);
+  p.num_blocks = num_blocks;
+  p.max_pages = max_pages;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.M = M;
+  p.causal = causal ? 1 : 0;
+  p.num_parts = num_sm_parts;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.timeout_ns = kDefaultTimeoutNs;
+
+  const uint64_t rows = static_cast<uint64_t>(num_blocks) * kPage;
+  CUtensorMap tm_a, tm_b;
+  cudaError_t e;
+  if (fmt == MLA_KV_BF16) {
+    if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_cache, kDqk, rows, kDqk * 2, 64, kPage,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_cache, kDqk, rows, kDqk * 2, 32, kPage,
+                  CU_TENSOR_MAP_SWIZZLE_64B))
+      return MLA_ERR_CUDA;
+    e = launch_decode_bf16(tm_a, tm_b, p, num_sm_parts, s);
+  } else {
+    // raw bytes: the latent half (256 B) of a token, and its 144-byte tail (scales + RoPE)
+    if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 256, kPage,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 144, kPage,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MLA_ERR_CUDA;
+    e = launch_decode_fp8(tm_a, tm_b, p, num_sm_parts, s);
+  }
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+
+  CombineParams c{};
+  c.sched = sched;
+  c.num_splits = num_splits;
+  c.lse_part = p.lse_part;
+  c.o_part = p.o_part;
+  c.out = p.out;
+  c.lse = lse;
+  c.batch = batch;
+  c.M = M;
+  c.num_parts = num_sm_parts;
+  e = launch_combine(c, num_sm_parts, s);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_last_device_status(const void* workspace, void* stream) {
+  if (!workspace) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  switch (status) {
+    case 0: return MLA_OK;
+    case kStatusBadSchedule: return MLA_ERR_INVALID_ARG;
+    case kStatusTimeout: return MLA_ERR_TIMEOUT;
+    case kStatusBadBlock: return MLA_ERR_BAD_BLOCK_INDEX;
+    default: return MLA_ERR_CUDA;
+  }
+}
+
+mla_status_t mla_clear_device_status(void* workspace, void* stream) {
+  if (!workspace) return MLA_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, sizeof(int), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+}  // extern "C"

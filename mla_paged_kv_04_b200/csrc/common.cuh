@@ -1,0 +1,99 @@
+// Shared definitions of the CUDA side: problem constants, the schedule
+// layout written by the metadata kernel, kernel parameter blocks and the
+// device-side error reporting.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+namespace mla {
+
+constexpr int kPage = 64;         // tokens per cache block
+constexpr int kDqk = 576;         // key width: 512 latent + 64 RoPE
+constexpr int kDv = 512;          // value width (the latent)
+constexpr int kDRope = 64;
+constexpr int kRows = 128;        // MMA M: query rows (s_q * h_q, padded) per work item
+constexpr int kFp8TokenBytes = 656;
+
+// Per-request fixed cost of the split-KV schedule, in units of one page.
+// A split costs a partial-output write plus its read-back in the combine
+// kernel (2 x 128 rows x 512 x 4 B, about 7 bf16 pages of traffic for a
+// 128-row request); a smaller value splits more eagerly.
+constexpr int kSplitOverheadPages = 4;
+
+// Schedule buffer (int32) written by the metadata kernel:
+//   [0] num_parts  [1] total_items  [2] units per part  [3] batch
+//   [4] overhead   [5] number of split requests  [6..8) reserved
+//   [8, 8 + num_parts + 1)          first item index of each part
+//   then num_parts ints             ids of the split requests (first [5] valid)
+//   then (16-byte aligned) 4 ints per item: request b, first page, end page, slot
+// Items are ordered by (request, split).  `slot` is the item's index when
+// the request is split (its partial-output row block), -1 otherwise.
+constexpr int kSchedHeader = 8;
+__host__ __device__ inline int sched_split_list_offset(int parts) { return kSchedHeader + parts + 1; }
+__host__ __device__ inline int sched_items_offset(int parts) {
+  return (sched_split_list_offset(parts) + parts + 3) & ~3;
+}
+__host__ __device__ inline size_t sched_ints(int batch, int parts) {
+  return static_cast<size_t>(sched_items_offset(parts)) +
+         4ull * (static_cast<size_t>(batch) + static_cast<size_t>(parts));
+}
+__host__ __device__ inline int max_items(int batch, int parts) { return batch + parts; }
+
+// Workspace: a 256-byte header (status word at offset 0), then fp32 partial
+// lse [max_items][M] and fp32 partial outputs [max_items][M][512].
+constexpr size_t kWsHeader = 256;
+__host__ __device__ inline size_t ws_lse_offset() { return kWsHeader; }
+__host__ __device__ inline size_t ws_o_offset(int batch, int parts, int M) {
+  size_t lse_bytes = 4ull * static_cast<size_t>(max_items(batch, parts)) * static_cast<size_t>(M);
+  return kWsHeader + ((lse_bytes + 255) / 256) * 256;
+}
+__host__ __device__ inline size_t ws_bytes(int batch, int parts, int M) {
+  return ws_o_offset(batch, parts, M) +
+         4ull * static_cast<size_t>(max_items(batch, parts)) * static_cast<size_t>(M) * kDv;
+}
+
+struct DecodeParams {
+  const uint16_t* q;            // bf16 [batch, M, 576]
+  const int32_t* block_table;   // [batch, max_pages]
+  const int32_t* seqlens;       // [batch]
+  const int32_t* sched;         // schedule buffer
+  uint16_t* out;                // bf16 [batch, M, 512]
+  float* lse;                   // [batch, M]
+  float* lse_part;              // [max_items, M]
+  float* o_part;                // [max_items, M, 512]
+  int* status;                  // workspace status word
+  long long num_blocks;
+  int max_pages;
+  int batch;
+  int s_q;
+  int h_q;
+  int M;
+  int causal;
+  int num_parts;                // CTA pairs launched (must equal sched[0])
+  float scale_log2;             // softmax_scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct CombineParams {
+  const int32_t* sched;         // schedule buffer (split-request list)
+  const int32_t* num_splits;    // [batch + 1]
+  const float* lse_part;
+  const float* o_part;
+  uint16_t* out;
+  float* lse;
+  int batch;
+  int M;
+  int num_parts;
+};
+
+// Status codes as stored in the workspace status word (match mla_status_t).
+constexpr int kStatusBadSchedule = 1;
+constexpr int kStatusTimeout = 5;
+constexpr int kStatusBadBlock = 6;
+
+__device__ __forceinline__ void report_status(int* status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+}  // namespace mla

@@ -1,0 +1,568 @@
+// MLA decode over a paged KV cache on sm_100a.
+//
+// Design (one CTA pair per "part" of the split-KV schedule, persistent over
+// the part's work items):
+//   * The two CTAs of a cluster split the 576 key dims: CTA r owns latent dims
+//     [256 r, 256 r + 256) and RoPE dims [512 + 32 r, 512 + 32 r + 32).  Each
+//     CTA gathers only its half of every 64-token page (block_table-driven TMA
+//     loads, 36 KB per page half), so KV crosses HBM once.
+//   * Q (this CTA's 288 dims, up to 128 query rows = s_q * h_q) lives in
+//     tensor memory and is the A operand of S_r = Q_r K_r^T, a tcgen05.mma
+//     with M = 128, N = 64 tokens, K = 288, accumulating fp32 in TMEM.
+//   * The pair swaps its partial S through distributed shared memory
+//     (st.async with transaction-count mbarriers) and both add them in the
+//     same order, so both CTAs hold the identical full S and take identical
+//     softmax decisions.
+//   * Online softmax in the log2 domain with a lazy rescale: the reference max
+//     only moves when the row max grows by more than 8 (a factor 256), so O
+//     is rescaled rarely.  P (bf16) is written to tensor memory.
+//   * O_r += P V_r with V_r = this CTA's latent half of the same smem page
+//     (the value is the first 512 dims of the key), M = 128, N = 256, K = 64,
+//     P taken from tensor memory, V as an MN-major operand of the same
+//     128-byte-swizzled tile the QK^T product read as K-major.
+//   * Epilogue: bf16 out and lse for an unsplit request, fp32 partials for a
+//     split one (merged by the combine kernel).
+//
+// Warp roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer,
+// warp 2 = tensor-memory allocator, warp 3 idle, warps 4-7 = softmax and
+// epilogue (thread r of the group owns query row r = tensor-memory lane r).
+//
+// Every wait on an mbarrier is bounded (params.timeout_ns); a wait that runs
+// out records MLA_ERR_TIMEOUT in the status word, raises a CTA-wide abort
+// flag and the CTA drains its copies and MMAs, frees tensor memory and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+
+namespace dk {
+constexpr int kChunkBytes = kPage * 128;                 // 64 tokens x 64 dims bf16 (SW128)
+constexpr int kRopeBytes = kPage * 64;                   // 64 tokens x 32 dims bf16 (SW64)
+constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;  // 36864: one page half
+constexpr int kXBytes = kRows * kPage * 4;              // 32768: one partial S tile
+constexpr int kRawLatBytes = kPage * 256;               // FP8: this CTA's 256 latent codes per token
+constexpr int kRawTailBytes = kPage * 144;              // FP8: 4 scales + 64 RoPE bf16 per token
+constexpr int kRawBytes = kRawLatBytes + kRawTailBytes; // 25600
+constexpr int kRawStages = 2;
+
+template <bool kFp8>
+struct Cfg {
+  static constexpr int kStages = kFp8 ? 3 : 4;           // bf16 page-half stages
+  static constexpr int kThreads = kFp8 ? 384 : 256;
+  // barrier indices
+  static constexpr int kFull = 0;
+  static constexpr int kEmpty = kFull + kStages;
+  static constexpr int kSFull = kEmpty + kStages;
+  static constexpr int kSFree = kSFull + 1;
+  static constexpr int kPFull = kSFree + 1;
+  static constexpr int kPvDone = kPFull + 1;
+  static constexpr int kQReady = kPvDone + 1;
+  static constexpr int kXFull = kQReady + 1;  // two
+  static constexpr int kDrain = kXFull + 2;
+  static constexpr int kRawFull = kDrain + 1;           // FP8 only
+  static constexpr int kRawEmpty = kRawFull + kRawStages;
+  static constexpr int kNumBars = kRawEmpty + kRawStages;
+  static constexpr int kRawOffset = kStages * kStageBytes + 2 * kXBytes;
+  static constexpr int kBarOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
+  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;
+};
+// tensor-memory columns (512 allocated)
+constexpr uint32_t kColO = 0;     // 256 fp32 columns: this CTA's half of O
+constexpr uint32_t kColS = 256;   // 64 fp32 columns: partial S
+constexpr uint32_t kColP = 320;   // 32 columns: P as packed bf16 pairs
+constexpr uint32_t kColQ = 352;   // 144 columns: Q (288 bf16) as packed pairs
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+}  // namespace dk
+
+__device__ const int g_never_abort = 0;
+
+// Warp-uniform bounded wait: lane 0 polls with the time limit, then every
+// lane performs its own (immediately successful) acquire of the same phase.
+template <bool kCluster = false>
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(bar, parity, abort, limit);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) {
+#pragma unroll 1
+    for (int i = 0; i < (1 << 20); ++i)
+      if (kCluster ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity)) break;
+  }
+  return ok != 0;
+}
+
+__device__ __forceinline__ void raise_abort(const DecodeParams& p, volatile int* abort_flag) {
+  report_status(p.status, kStatusTimeout);
+  *abort_flag = 1;
+}
+
+
+// 16 E4M3 codes (one 16-byte raw unit) times an fp32 scale -> 16 bf16 (RNE),
+// as 8 packed pairs in memory order.  e4m3 -> f16 is exact; the product is
+// formed in fp32 and rounded once to bf16.
+__device__ __forceinline__ void dequant16(const uint4 raw, float sc, uint32_t (&w)[8]) {
+  const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((in[i] >> (16 * h)) & 0xFFFFu);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float lo = __half2float(__ushort_as_half(hr.x));
+      const float hi = __half2float(__ushort_as_half(hr.y));
+      w[2 * i + h] = pack_bf16x2(lo * sc, hi * sc);
+    }
+  }
+}
+
+template <bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                  const DecodeParams p) {
+  using namespace dk;
+  using C = Cfg<kFp8>;
+  constexpr int kStages = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw_addr);
+  const uint32_t stage0 = base;
+  const uint32_t xbuf0 = base + kStages * kStageBytes;
+  const uint32_t rawbuf0 = base + C::kRawOffset;
+  const uint32_t bar0 = base + C::kBarOffset;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::kBarOffset + C::kNumBars * 8);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sbase + C::kBarOffset + C::kNumBars * 8 + 4);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int part = static_cast<int>(cluster_id_x());
+  const int num_parts = p.sched[0];
+  const int32_t* items = p.sched + sched_items_offset(num_parts);
+  int it_begin = 0, it_end = 0;
+  if (num_parts != p.num_parts) {
+    // schedule made for another CTA-pair count: its item slots may not fit
+    // the workspace, so do nothing and report it
+    if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
+  } else {
+    it_begin = p.sched[kSchedHeader + part];
+    it_end = p.sched[kSchedHeader + part + 1];
+  }
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(BAR(C::kFull + i), kFp8 ? 4 : 1);  // FP8: the four dequant warps arrive
+      mbar_init(BAR(C::kEmpty + i), 1);
+    }
+    mbar_init(BAR(C::kSFull), 1);
+    mbar_init(BAR(C::kSFree), 4);
+    mbar_init(BAR(C::kPFull), 4);
+    mbar_init(BAR(C::kPvDone), 1);
+    mbar_init(BAR(C::kQReady), 4);
+    mbar_init(BAR(C::kXFull), 1);
+    mbar_init(BAR(C::kXFull + 1), 1);
+    mbar_init(BAR(C::kDrain), 1);
+    for (int i = 0; i < kRawStages; ++i) {
+      mbar_init(BAR(C::kRawFull + i), 1);
+      mbar_init(BAR(C::kRawEmpty + i), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  cluster_sync();  // the peer's barriers are initialised before any st.async reaches them
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      // BF16: page halves straight into the MMA stages.  FP8: raw bytes into
+      // the raw stages, for the dequant warps.
+      constexpr int nst = kFp8 ? kRawStages : kStages;
+      const int full0 = kFp8 ? C::kRawFull : C::kFull;
+      const int empty0 = kFp8 ? C::kRawEmpty : C::kEmpty;
+      uint32_t g = 0;
+      bool ok = true;
+      for (int it = it_begin; it < it_end && ok; ++it) {
+        const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
+        const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
+        for (int pg = p0; pg < p1; ++pg, ++g) {
+          const uint32_t st = g % nst;
+          if (g >= static_cast<uint32_t>(nst) &&
+              !mbar_wait(BAR(empty0 + st), ((g / nst) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+            raise_abort(p, abort_flag);
+            ok = false;
+            break;
+          }
+          // A page past the block table's row (cache_seqlens larger than
+          // 64 * max_pages) is treated like a bad block index.
+          long long phys = pg < p.max_pages ? bt[pg] : -1;
+          if (phys < 0 || phys >= p.num_blocks) {
+            report_status(p.status, kStatusBadBlock);
+            phys = 0;
+          }
+          const int y = static_cast<int>(phys) * kPage;
+          const uint32_t fb = BAR(full0 + st);
+          if constexpr (kFp8) {
+            const uint32_t dst = rawbuf0 + st * kRawBytes;
+            mbar_arrive_expect_tx(fb, kRawBytes);
+            tma_load_2d(dst, &tm_a, fb, static_cast<int>(rank) * 256, y);
+            tma_load_2d(dst + kRawLatBytes, &tm_b, fb, 512, y);
+          } else {
+            const uint32_t dst = stage0 + st * kStageBytes;
+            mbar_arrive_expect_tx(fb, kStageBytes);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(dst + c * kChunkBytes, &tm_a, fb, static_cast<int>(rank) * 256 + c * 64, y);
+            tma_load_2d(dst + 4 * kChunkBytes, &tm_b, fb, 512 + static_cast<int>(rank) * 32, y);
+          }
+        }
+      }
+      // Never leave a copy landing in shared memory after the CTA exits.
+      for (uint32_t k = (g > static_cast<uint32_t>(nst) ? g - nst : 0u); k < g; ++k)
+        mbar_wait(BAR(full0 + k % nst), (k / nst) & 1u, &g_never_abort, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
+      uint32_t g = 0, nitem = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+        if (!mbar_wait(BAR(C::kPFull), gg & 1u, abort_flag, p.timeout_ns)) return false;
+        tc_fence_after();
+        const uint32_t sb = stage0 + (gg % kStages) * kStageBytes;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bd = sdesc(sb + ks * 2048, 8192, 1024, kSwizzle128);
+          mma_ts(tmem + kColO, tmem + kColP + ks * 8, bd, idesc_pv, (first && ks == 0) ? 0u : 1u);
+        }
+        tc_commit(BAR(C::kPvDone));
+        tc_commit(BAR(C::kEmpty + gg % kStages));
+        return true;
+      };
+      for (int it = it_begin; it < it_end && ok; ++it) {
+        const int n = items[4 * it + 2] - items[4 * it + 1];
+        if (n <= 0) continue;
+        if (!mbar_wait(BAR(C::kQReady), nitem & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        ++nitem;
+        tc_fence_after();
+        for (int j = 0; j < n; ++j, ++g) {
+          const uint32_t st = g % kStages;
+          if (!mbar_wait(BAR(C::kFull + st), (g / kStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          if (g > 0 && !mbar_wait(BAR(C::kSFree), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sb = stage0 + st * kStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < 18; ++ks) {
+            const uint64_t bd = ks < 16 ? sdesc(sb + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024, kSwizzle128)
+                                        : sdesc(sb + 4 * kChunkBytes + (ks - 16) * 32, 16, 512, kSwizzle64);
+            mma_ts(tmem + kColS, tmem + kColQ + ks * 8, bd, idesc_qk, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(BAR(C::kSFull));
+          if (j > 0 && !issue_pv(g - 1, j == 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!issue_pv(g - 1, n == 1)) { ok = false; break; }
+      }
+      if (!ok) raise_abort(p, abort_flag);
+      // All issued MMAs complete before tensor memory is released.
+      tc_commit(BAR(C::kDrain));
+      mbar_wait(BAR(C::kDrain), 0, &g_never_abort, 100000000ull);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int wq = warp - 4;
+    const int r = threadIdx.x - 128;  // query row == tensor-memory lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t xpeer = mapa_shared(xbuf0, peer);
+    const uint32_t xbar_peer = mapa_shared(BAR(C::kXFull), peer);
+    const float4* xlocal = reinterpret_cast<const float4*>(sbase + kStages * kStageBytes);
+    uint32_t g = 0;
+    bool ok = true;
+    const bool row_ok = r < p.M;
+    const int qi = r / p.h_q;
+    for (int it = it_begin; it < it_end && ok; ++it) {
+      const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2], slot = items[4 * it + 3];
+      const int L = p.seqlens[b];
+      const int n = p1 - p0;
+      const size_t orow = static_cast<size_t>(b) * p.M + r;
+      if (n <= 0) {
+        if (row_ok) {
+          if (slot >= 0) {
+            if (rank == 0) p.lse_part[static_cast<size_t>(slot) * p.M + r] = -CUDART_INF_F;
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256);
+            for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+            if (rank == 0) p.lse[orow] = -CUDART_INF_F;
+          }
+        }
+        continue;
+      }
+      // Q -> tensor memory (this CTA's 288 dims as 144 packed bf16 pairs).
+      {
+        const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow * kDqk);
+#pragma unroll 1
+        for (int c16 = 0; c16 < 9; ++c16) {
+          uint32_t v[16];
+          const int e0 = (c16 < 8) ? static_cast<int>(rank) * 256 + c16 * 32 : 512 + static_cast<int>(rank) * 32;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 w = row_ok ? __ldg(qrow + e0 / 8 + u) : make_uint4(0, 0, 0, 0);
+            v[4 * u + 0] = w.x;
+            v[4 * u + 1] = w.y;
+            v[4 * u + 2] = w.z;
+            v[4 * u + 3] = w.w;
+          }
+          tmem_st16(trow + kColQ + c16 * 16, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::kQReady));
+      }
+      const int vis = p.causal ? min(L, L - p.s_q + qi + 1) : L;
+      const int last_page = (L - 1) / kPage;
+      float m_ref = -CUDART_INF_F, l = 0.f;
+      for (int j = 0; j < n; ++j, ++g) {
+        const int pg = p0 + j;
+        if (!warp_wait(BAR(C::kSFull), g & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t s[64];
+        tmem_ld32(trow + kColS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(trow + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::kSFree));
+        // swap partial S with the peer CTA
+        const uint32_t xb = g & 1u;
+        if (r == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXBytes);
+        {
+          const uint32_t rx = xpeer + xb * kXBytes;
+          const uint32_t rbar = xbar_peer + 8u * xb;
+#pragma unroll
+          for (int c4 = 0; c4 < 16; ++c4)
+            st_async_v4(rx + (c4 * 128 + r) * 16, __uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1]),
+                        __uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3]), rbar);
+        }
+        if (!warp_wait<true>(BAR(C::kXFull + xb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        float x[64];
+        float mt = -CUDART_INF_F;
+        const int tok0 = pg * kPage;
+        const float4* xs = xlocal + xb * (kXBytes / 16);
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 pv = xs[c4 * 128 + r];
+          const float pe[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = 4 * c4 + e;
+            float v = (__uint_as_float(s[t]) + pe[e]) * p.scale_log2;
+            v = (tok0 + t < vis) ? v : -CUDART_INF_F;
+            x[t] = v;
+            mt = fmaxf(mt, v);
+          }
+        }
+        const float m_new = fmaxf(m_ref, mt);
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        const float m_use = need ? m_new : m_ref;
+        const float m_sub = (m_use == -CUDART_INF_F) ? 0.f : m_use;
+        uint32_t pk[32];
+        float rowsum = 0.f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          const float a = ex2_approx(x[2 * t] - m_sub);
+          const float c = ex2_approx(x[2 * t + 1] - m_sub);
+          pk[t] = pack_bf16x2(a, c);
+          rowsum += a + c;  // fp32 probabilities: the bf16 rounding of P must not reach lse
+        }
+        // The previous tile's PV must be done: P is single-buffered and O may be rescaled.
+        if (g > 0) {
+          if (!warp_wait(BAR(C::kPvDone), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+        }
+        const float factor = need ? ex2_approx(m_ref - m_use) : 1.f;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(trow + kColO + cc * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            tmem_st16(trow + kColO + cc * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+            tmem_st16(trow + kColO + cc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+          }
+        }
+        l = l * factor + rowsum;
+        m_ref = m_use;
+        if constexpr (!kFp8) {
+          // Slots past the end of the request on its last page may hold NaN/Inf:
+          // zero those V rows so that 0 * garbage cannot reach O.  (The FP8
+          // dequant warps write zeros there themselves.)
+          if (pg == last_page && (L & (kPage - 1))) {
+            const int t0 = L & (kPage - 1);
+            uint8_t* stg = sbase + (g % kStages) * kStageBytes;
+            for (int u = r; u < (kPage - t0) * 32; u += 128) {
+              const int row = t0 + (u >> 5), w = u & 31;
+              *reinterpret_cast<uint4*>(stg + (w >> 3) * kChunkBytes + row * 128 + (w & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
+        }
+        tmem_st16(trow + kColP, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(trow + kColP + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::kPFull));
+      }
+      if (!ok) break;
+      // epilogue
+      if (!warp_wait(BAR(C::kPvDone), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse_val = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+#pragma unroll 1
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(trow + kColO + cc * 32, o);
+        if (row_ok) {
+          if (slot < 0) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256 + cc * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
+                                  pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(slot) * p.M + r) * kDv +
+                                                    rank * 256 + cc * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                   __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+          }
+        }
+      }
+      if (row_ok && rank == 0) {
+        if (slot < 0) p.lse[orow] = lse_val;
+        else p.lse_part[static_cast<size_t>(slot) * p.M + r] = lse_val;
+      }
+    }
+    if (!ok) raise_abort(p, abort_flag);
+  } else if (kFp8 && warp >= 8) {
+    // ------------------------------------------------------------------ FP8 dequant (warps 8-11)
+    // Raw 656-byte tokens -> this CTA's bf16 page half, in the same swizzled
+    // layout the BF16 path gets from TMA.  Thread dt handles 16-code units
+    // u = dt + 128 k: token u / 16, codes 16 (u % 16) .. +16 of the CTA's 256.
+    const int dt = threadIdx.x - 256;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int it = it_begin; it < it_end && ok; ++it) {
+      const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
+      const int L = p.seqlens[b];
+      const int last_page = (L - 1) / kPage;
+      for (int pg = p0; pg < p1; ++pg, ++g) {
+        const uint32_t rs = g % kRawStages, st = g % kStages;
+        if (!warp_wait(BAR(C::kRawFull + rs), (g / kRawStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (g >= static_cast<uint32_t>(kStages) &&
+            !warp_wait(BAR(C::kEmpty + st), ((g / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const int valid = (pg == last_page) ? L - pg * kPage : kPage;
+        const uint8_t* rlat = sbase + C::kRawOffset + rs * kRawBytes;
+        const uint8_t* rtail = rlat + kRawLatBytes;
+        uint8_t* dst = sbase + st * kStageBytes;
+#pragma unroll 2
+        for (int k = 0; k < 8; ++k) {
+          const int u = dt + 128 * k;
+          const int t = u >> 4, g16 = u & 15;
+          uint32_t w[8];
+          if (t < valid) {
+            const uint4 codes = *reinterpret_cast<const uint4*>(rlat + t * 256 + g16 * 16);
+            const float sc = *reinterpret_cast<const float*>(rtail + t * 144 + 4 * (2 * static_cast<int>(rank) + (g16 >> 3)));
+            dequant16(codes, sc, w);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = 0u;
+          }
+          uint8_t* row = dst + (g16 >> 2) * kChunkBytes + t * 128;
+          const int u0 = (g16 & 3) * 2;
+          *reinterpret_cast<uint4*>(row + ((u0 ^ (t & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(row + (((u0 + 1) ^ (t & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int u = dt + 128 * k;
+          const int t = u >> 2, w4 = u & 3;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (t < valid) v = *reinterpret_cast<const uint4*>(rtail + t * 144 + 16 + static_cast<int>(rank) * 64 + w4 * 16);
+          *reinterpret_cast<uint4*>(dst + 4 * kChunkBytes + t * 64 + ((w4 ^ ((t >> 1) & 3)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(BAR(C::kFull + st));
+          mbar_arrive(BAR(C::kRawEmpty + rs));
+        }
+      }
+    }
+    if (!ok) raise_abort(p, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer no longer writes into this CTA's exchange buffers
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+#undef BAR
+}
+
+template <bool kFp8>
+static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const DecodeParams& p,
+                                 int num_parts, cudaStream_t stream) {
+  using C = dk::Cfg<kFp8>;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  decode_kernel<kFp8><<<2 * num_parts, C::kThreads, C::kSmemBytes, stream>>>(tm_a, tm_b, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
+                               int num_parts, cudaStream_t stream) {
+  return launch_decode<false>(tm_lat, tm_rope, p, num_parts, stream);
+}
+
+cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_tail, const DecodeParams& p,
+                              int num_parts, cudaStream_t stream) {
+  return launch_decode<true>(tm_lat, tm_tail, p, num_parts, stream);
+}
+
+}  // namespace mla

@@ -1,0 +1,167 @@
+// Split-KV schedule for variable-length batches, computed on the device by a
+// single 1024-thread block so that it stays on the caller's stream.
+//
+// Cost model: request b costs n_b + c units, n_b = ceil(L_b / 64) pages and
+// c = kSplitOverheadPages.  The requests' cost intervals are laid end to end
+// (exclusive prefix C_b) and the line [0, T) is cut into pieces of
+// t = ceil(T / parts) units; piece k belongs to CTA pair ("part") k.  A
+// request crossing a cut is split there: split s of request b covers the
+// virtual range [max(C_b, k t), min(C_b + cost_b, (k + 1) t)) - C_b with
+// k = floor(C_b / t) + s; the first c virtual units of a request stand for
+// its fixed cost, so virtual position v maps to page clamp(v - c, 0, n_b).
+// A split may therefore hold zero pages; the decode kernel then only writes
+// lse = -inf for it and the combine kernel gives it no weight.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+constexpr int kMetaThreads = 1024;
+constexpr int kMaxBatch = 16384;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < (kMetaThreads / 32)) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  int prefix = x - v + (warp > 0 ? warp_sums[warp - 1] : 0);
+  *total = warp_sums[kMetaThreads / 32 - 1];
+  __syncthreads();
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
+                                                                int parts, int overhead, int32_t* __restrict__ sched,
+                                                                int32_t* __restrict__ num_splits) {
+  extern __shared__ int sm[];
+  int* C = sm;                 // [batch + 1] cost prefix
+  int* S = sm + batch + 1;     // [batch + 1] split prefix
+  __shared__ int warp_sums[32];
+
+  const int per = (batch + kMetaThreads - 1) / kMetaThreads;
+  const int b0 = threadIdx.x * per;
+  const int b1 = min(batch, b0 + per);
+
+  // 1. cost prefix
+  int local = 0;
+  for (int b = b0; b < b1; ++b) {
+    int L = max(seqlens[b], 0);
+    local += (L + kPage - 1) / kPage + overhead;
+  }
+  int T;
+  int run = block_exclusive_scan(local, warp_sums, &T);
+  for (int b = b0; b < b1; ++b) {
+    C[b] = run;
+    int L = max(seqlens[b], 0);
+    run += (L + kPage - 1) / kPage + overhead;
+  }
+  if (threadIdx.x == 0) C[batch] = T;
+  __syncthreads();
+  const int t = max(1, (T + parts - 1) / parts);
+
+  // 2. splits per request and their prefix
+  local = 0;
+  for (int b = b0; b < b1; ++b) {
+    int k0 = C[b] / t, k1 = (C[b + 1] - 1) / t;
+    local += k1 - k0 + 1;
+  }
+  int I;
+  run = block_exclusive_scan(local, warp_sums, &I);
+  for (int b = b0; b < b1; ++b) {
+    S[b] = run;
+    int k0 = C[b] / t, k1 = (C[b + 1] - 1) / t;
+    run += k1 - k0 + 1;
+  }
+  if (threadIdx.x == 0) S[batch] = I;
+  __syncthreads();
+
+  // 3. items, and the compact list of split requests
+  int32_t* part_first = sched + kSchedHeader;
+  int32_t* split_list = sched + sched_split_list_offset(parts);
+  int32_t* items = sched + sched_items_offset(parts);
+  local = 0;
+  for (int b = b0; b < b1; ++b) local += ((C[b + 1] - 1) / t - C[b] / t) > 0;
+  int nsplit_req;
+  int split_pos = block_exclusive_scan(local, warp_sums, &nsplit_req);
+  for (int b = b0; b < b1; ++b) {
+    const int L = max(seqlens[b], 0);
+    const int n = (L + kPage - 1) / kPage;
+    const int cb = C[b], cost = C[b + 1] - C[b];
+    const int k0 = cb / t, k1 = (C[b + 1] - 1) / t;
+    const int K = k1 - k0 + 1;
+    for (int s = 0; s < K; ++s) {
+      const int k = k0 + s;
+      const int v0 = max(cb, k * t) - cb;
+      const int v1 = min(cb + cost, (k + 1) * t) - cb;
+      const int p0 = min(max(v0 - overhead, 0), n);
+      const int p1 = min(max(v1 - overhead, 0), n);
+      const int idx = S[b] + s;
+      items[4 * idx + 0] = b;
+      items[4 * idx + 1] = p0;
+      items[4 * idx + 2] = p1;
+      items[4 * idx + 3] = (K > 1) ? idx : -1;
+    }
+    if (K > 1) split_list[split_pos++] = b;
+    num_splits[b] = S[b];
+  }
+  if (threadIdx.x == 0) {
+    num_splits[batch] = I;
+    sched[0] = parts;
+    sched[1] = I;
+    sched[2] = t;
+    sched[3] = batch;
+    sched[4] = overhead;
+    sched[5] = nsplit_req;
+    sched[6] = sched[7] = 0;
+  }
+
+  // 4. first item of each part: the request holding virtual position k t
+  for (int k = threadIdx.x; k <= parts; k += blockDim.x) {
+    const long long pos = static_cast<long long>(k) * t;
+    int first;
+    if (k == parts || pos >= T) {
+      first = I;
+    } else {
+      int lo = 0, hi = batch - 1;  // largest b with C[b] <= pos
+      while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (C[mid] <= pos) lo = mid; else hi = mid - 1;
+      }
+      first = S[lo] + (k - C[lo] / t);
+    }
+    part_first[k] = first;
+  }
+}
+
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int parts, int32_t* sched, int32_t* num_splits,
+                            cudaStream_t stream) {
+  const size_t smem = 2ull * (batch + 1) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, parts, kSplitOverheadPages, sched,
+                                                     num_splits);
+  return cudaGetLastError();
+}
+
+int metadata_max_batch() { return kMaxBatch; }
+
+}  // namespace mla

@@ -1,0 +1,80 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path, run the oracle,
+and compare with the tolerances of the method's accuracy contract:
+  out: max |err| <= 2e-2 and mean |err| <= 2e-3  (bf16 output vs float64)
+  lse: max |err| <= 1e-3
+"""
+
+import numpy as np
+import torch
+
+import oracle
+import workloads as W
+
+OUT_MAX_TOL = 2e-2
+OUT_MEAN_TOL = 2e-3
+LSE_TOL = 1e-3
+
+
+def run_gpu(case, num_sm_parts=None, workspace=None):
+    import mla_paged_kv_04_b200 as mla
+    dev = torch.device("cuda")
+    q = case["q"].to(dev)
+    kv = case["kv_cache"].to(dev)
+    bt = case["block_table"].to(dev)
+    L = case["cache_seqlens"].to(dev)
+    B, s_q, h_q, _ = q.shape
+    parts = mla.mla_default_num_sm_parts() if num_sm_parts is None else num_sm_parts
+    sched, ns = mla.mla_get_metadata(L, s_q, h_q, parts)
+    ws = mla.alloc_workspace(B, s_q, h_q, parts, dev) if workspace is None else workspace
+    out = torch.empty((B, s_q, h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    mla.mla_decode_fwd(q, kv, case["fmt"], bt, L, case["softmax_scale"], case["causal"], sched, ns, parts,
+                       out, lse, ws)
+    status = mla.mla_last_device_status(ws)
+    return out.float().cpu().double().numpy(), lse.cpu().double().numpy(), status
+
+
+def fp8_cache_as_bf16(kv_u8: torch.Tensor) -> torch.Tensor:
+    """The dequantised cache the kernel computes on: bf16(fp32(e4m3) * fp32(scale)).
+
+    Test-side input preparation (torch on CPU) so that the FP8 parity check can
+    feed the oracle "the same dequantised cache" as the GPU path.
+    """
+    kv = kv_u8.cpu()
+    nb = kv.shape[0]
+    flat = kv.reshape(-1, 656)
+    codes = flat[:, :512].contiguous().view(torch.float8_e4m3fn).float()
+    scales = flat[:, 512:528].contiguous().view(torch.float32)
+    lat = (codes.view(-1, 4, 128) * scales[:, :, None]).view(-1, 512).to(torch.bfloat16)
+    rope = flat[:, 528:].contiguous().view(torch.bfloat16)
+    return torch.cat([lat, rope], dim=1).view(nb, 64, 576)
+
+
+def oracle_for(case, requests=None, dequant_bf16=False):
+    """Oracle (float64) outputs for all or some requests of a case."""
+    if dequant_bf16 and case["fmt"] == "fp8_656":
+        case = dict(case)
+        case["kv_cache"] = fp8_cache_as_bf16(case["kv_cache"])
+        case["fmt"] = "bf16"
+    if requests is None:
+        a = W.oracle_arrays(case)
+        return oracle.mla_decode(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
+                                 a["softmax_scale"], a["causal"])
+    a = W.oracle_arrays_for(case, requests)
+    res = oracle.mla_decode_rows(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
+                                 a["softmax_scale"], a["causal"], requests)
+    return res
+
+
+def check(out, lse, ref_out, ref_lse, what=""):
+    """Element-wise comparison; -inf lse must match exactly (empty rows)."""
+    err = np.abs(out - ref_out)
+    assert np.all(np.isfinite(out)), f"{what}: non-finite output"
+    assert err.max() <= OUT_MAX_TOL, f"{what}: out max err {err.max():.3g}"
+    assert err.mean() <= OUT_MEAN_TOL, f"{what}: out mean err {err.mean():.3g}"
+    inf_ref = np.isneginf(ref_lse)
+    assert np.array_equal(np.isneginf(lse), inf_ref), f"{what}: -inf lse pattern differs"
+    if (~inf_ref).any():
+        lerr = np.abs(lse[~inf_ref] - ref_lse[~inf_ref])
+        assert lerr.max() <= LSE_TOL, f"{what}: lse max err {lerr.max():.3g}"
+    return float(err.max()), float(err.mean())

@@ -1,0 +1,101 @@
+"""The C-ABI shared library, without a GPU: it builds, loads, exports every
+entry point that include/mla.h declares, and rejects bad arguments with the
+documented status before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mla_paged_kv_04_b200 import build
+    build.build()
+    import mla_paged_kv_04_b200 as mla
+    return mla.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for required in ("mla_get_metadata", "mla_decode_fwd", "mla_workspace_size", "mla_metadata_size"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+def test_status_strings(lib):
+    import mla_paged_kv_04_b200 as mla
+    for code, name in mla.STATUS.items():
+        assert mla.mla_status_string(code) == name
+
+
+def test_sizes(lib):
+    import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import schedule
+    assert mla.mla_metadata_size(64, 74) == 4 * schedule.sched_ints(64, 74)
+    assert mla.mla_metadata_size(0, 74) == 0
+    w1 = mla.mla_workspace_size(64, 1, 128, 74)
+    w2 = mla.mla_workspace_size(64, 1, 128, 148)
+    assert w1 >= 256 + (64 + 74) * 128 * 513 * 4 and w2 > w1
+    assert mla.mla_workspace_size(1, 2, 128, 74) == 0  # M = 256 unsupported
+
+
+def _call_decode(lib, **over):
+    args = dict(q=16, kv=16, fmt=0, num_blocks=10, bt=16, max_pages=4, seqlens=16, batch=2, s_q=1, h_q=16,
+                scale=0.0417, causal=0, sched=16, ns=16, parts=74, out=16, lse=16, ws=256, ws_bytes=1 << 30,
+                stream=None)
+    args.update(over)
+    return lib.mla_decode_fwd(args["q"], args["kv"], args["fmt"], args["num_blocks"], args["bt"],
+                              args["max_pages"], args["seqlens"], args["batch"], args["s_q"], args["h_q"],
+                              args["scale"], args["causal"], args["sched"], args["ns"], args["parts"],
+                              args["out"], args["lse"], args["ws"], args["ws_bytes"], args["stream"])
+
+
+def test_decode_argument_validation(lib):
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+    assert _call_decode(lib, q=None) == INVALID
+    assert _call_decode(lib, kv=None) == INVALID
+    assert _call_decode(lib, q=8) == INVALID            # misaligned
+    assert _call_decode(lib, ws=128) == INVALID         # workspace not 256-aligned
+    assert _call_decode(lib, fmt=7) == INVALID
+    assert _call_decode(lib, num_blocks=0) == INVALID
+    assert _call_decode(lib, max_pages=0) == INVALID
+    assert _call_decode(lib, scale=float("nan")) == INVALID
+    assert _call_decode(lib, scale=float("inf")) == INVALID
+    assert _call_decode(lib, batch=0) == INVALID
+    assert _call_decode(lib, s_q=2, h_q=128) == UNSUPPORTED   # M = 256 > 128
+    assert _call_decode(lib, batch=20000) == UNSUPPORTED
+    assert _call_decode(lib, ws_bytes=1024) == WORKSPACE
+
+
+def test_metadata_argument_validation(lib):
+    INVALID, UNSUPPORTED = 1, 2
+    f = lib.mla_get_metadata
+    assert f(None, 4, 1, 128, 74, 16, 16, None) == INVALID
+    assert f(16, 4, 1, 128, 0, 16, 16, None) == INVALID
+    assert f(16, 4, 1, 128, 74, 8, 16, None) == INVALID   # sched must be 16-byte aligned
+    assert f(16, 0, 1, 128, 74, 16, 16, None) == INVALID
+    assert f(16, 4, 3, 64, 74, 16, 16, None) == UNSUPPORTED
+
+
+def test_product_has_no_oracle_dependency():
+    pkg = os.path.join(ROOT, "mla_paged_kv_04_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f

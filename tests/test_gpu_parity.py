@@ -1,0 +1,157 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small cases run the oracle on every output element; the five configured
+workloads run at full size in the launch configuration the bench times, with
+the oracle evaluated on sampled requests.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from _gpu_helpers import check, oracle_for, run_gpu, fp8_cache_as_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mla_paged_kv_04_b200 import build
+    build.build()
+    import mla_paged_kv_04_b200 as mla
+    mla.load_library()
+
+
+def _case(batch, s_q, h_q, seqlens, fmt="bf16", causal=False, seed=0, poison=True):
+    w = W.Workload("t", batch, s_q, h_q, (1, 1), fmt=fmt, causal=causal, seed=seed)
+    return W.make_case(w, seqlens=list(seqlens), poison=poison)
+
+
+def test_tiny_config_full():
+    c = W.make_case(W.WORKLOADS["tiny"])
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    ro, rl = oracle_for(c)
+    check(out, lse, ro, rl, "tiny")
+
+
+SMALL = [
+    # batch, s_q, h_q, seqlens, causal
+    (4, 1, 128, (300, 1000, 64, 130), False),
+    (3, 2, 64, (700, 1, 65), True),
+    (5, 1, 16, (63, 64, 65, 128, 1), False),
+    (2, 2, 32, (129, 2), True),
+    (2, 1, 100, (257, 190), False),   # M not a power of two
+    (2, 4, 32, (333, 4), True),       # s_q = 4
+]
+
+
+@pytest.mark.parametrize("batch,s_q,h_q,seqlens,causal", SMALL)
+def test_small_bf16(batch, s_q, h_q, seqlens, causal):
+    c = _case(batch, s_q, h_q, seqlens, causal=causal, seed=batch + s_q)
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    ro, rl = oracle_for(c)
+    check(out, lse, ro, rl, f"bf16 {seqlens}")
+
+
+@pytest.mark.parametrize("batch,s_q,h_q,seqlens,causal", SMALL[:4])
+def test_small_fp8(batch, s_q, h_q, seqlens, causal):
+    c = _case(batch, s_q, h_q, seqlens, fmt="fp8_656", causal=causal, seed=7 + batch)
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    ro, rl = oracle_for(c, dequant_bf16=True)
+    check(out, lse, ro, rl, f"fp8 {seqlens}")
+
+
+def test_fp8_against_exact_dequant_oracle():
+    # The exact e4m3*scale products (no bf16 rounding) stay within the same
+    # tolerances once requests hold more than a handful of tokens.
+    c = _case(3, 1, 128, (2000, 700, 4000), fmt="fp8_656", seed=3)
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    ro, rl = oracle_for(c)
+    check(out, lse, ro, rl, "fp8 exact")
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 7, 74, 200])
+def test_forced_splits_agree(parts):
+    c = _case(3, 2, 64, (1500, 100, 777), causal=True, seed=11)
+    out, lse, st = run_gpu(c, num_sm_parts=parts)
+    assert st == 0
+    ro, rl = oracle_for(c)
+    check(out, lse, ro, rl, f"parts={parts}")
+
+
+def test_zero_length_and_empty_causal_row():
+    c = _case(3, 2, 16, (0, 1, 70), causal=True, seed=2)
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    ro, rl = oracle_for(c)
+    check(out, lse, ro, rl, "empty rows")
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(out[1, 0] == 0) and np.all(np.isneginf(lse[1, 0]))
+
+
+def test_poison_does_not_change_results():
+    seqlens = (65, 200, 7)
+    clean = _case(3, 1, 64, seqlens, poison=False, seed=4)
+    dirty = _case(3, 1, 64, seqlens, poison=True, seed=4)
+    o1, l1, s1 = run_gpu(clean)
+    o2, l2, s2 = run_gpu(dirty)
+    assert s1 == 0 and s2 == 0
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_deterministic():
+    c = _case(2, 1, 128, (900, 300), seed=5)
+    o1, l1, _ = run_gpu(c, num_sm_parts=8)
+    o2, l2, _ = run_gpu(c, num_sm_parts=8)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_bad_block_index_reported():
+    import mla_paged_kv_04_b200 as mla
+    c = _case(2, 1, 16, (130, 64), seed=6)
+    c["block_table"][0, 1] = c["num_blocks"] + 5
+    out, lse, st = run_gpu(c)
+    assert mla.STATUS[st] == "MLA_ERR_BAD_BLOCK_INDEX"
+
+
+def test_metadata_covers_every_page_once():
+    import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import schedule
+    g = torch.Generator().manual_seed(9)
+    for parts in (1, 5, 74, 300):
+        L = torch.randint(0, 5000, (97,), generator=g, dtype=torch.int32)
+        L[3] = 0
+        sched, ns = mla.mla_get_metadata(L.cuda(), 1, 128, parts)
+        torch.cuda.synchronize()
+        dev_sched, dev_ns = sched.cpu().numpy(), ns.cpu().numpy()
+        schedule.validate(dev_sched, dev_ns, L.numpy(), parts)
+        host_sched, host_ns = schedule.plan(L.numpy(), parts)
+        np.testing.assert_array_equal(dev_ns, host_ns)
+        used = schedule.items_offset(parts) + 4 * int(host_sched[1])
+        np.testing.assert_array_equal(dev_sched[:8], host_sched[:8])
+        np.testing.assert_array_equal(dev_sched[8:8 + parts + 1], host_sched[8:8 + parts + 1])
+        io = schedule.items_offset(parts)
+        np.testing.assert_array_equal(dev_sched[io:used], host_sched[io:used])
+
+
+@pytest.mark.parametrize("name", W.ORDER)
+def test_full_size_sampled(name):
+    w = W.WORKLOADS[name]
+    c = W.make_case(w, device="cuda")
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    L = c["cache_seqlens"].cpu().numpy()
+    picks = sorted({0, int(np.argmax(L)), int(np.argmin(L)), w.batch - 1})
+    ref = oracle_for(c, picks, dequant_bf16=(w.fmt == "fp8_656"))
+    for b in picks:
+        check(out[b], lse[b], ref[b][0], ref[b][1], f"{name} request {b}")
+    assert np.all(np.isfinite(out))

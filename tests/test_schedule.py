@@ -1,0 +1,50 @@
+"""Host logic of the split-KV schedule (CPU only): the host planner produces
+valid plans (every page covered exactly once, items contiguous per part and
+per request, split bookkeeping consistent) across lengths and part counts."""
+
+import numpy as np
+import pytest
+
+from mla_paged_kv_04_b200 import schedule
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 7, 74, 148, 500])
+def test_plan_is_valid_random(parts):
+    rng = np.random.default_rng(parts)
+    for batch in (1, 2, 17, 128, 1000):
+        L = rng.integers(0, 9000, batch)
+        sched, ns = schedule.plan(L, parts)
+        schedule.validate(sched, ns, L, parts)
+
+
+def test_plan_edge_lengths():
+    for L in ([0], [1], [63, 64, 65], [0, 0, 0], [131072] * 8, [1] * 300):
+        for parts in (1, 5, 74):
+            sched, ns = schedule.plan(L, parts)
+            schedule.validate(sched, ns, L, parts)
+
+
+def test_long_context_is_split_across_parts():
+    # 8 requests of 2048 pages on 74 CTA pairs: every request is split ~9 ways
+    sched, ns = schedule.plan([131072] * 8, 74)
+    splits = np.diff(ns)
+    assert splits.min() >= 9 and int(sched[5]) == 8
+    loads = [sum(p1 - p0 for _, p0, p1, _ in part) for part in schedule.parse(sched, 74)]
+    assert max(loads) <= -(-8 * 2048 // 74) + 4  # within the per-request overhead of a perfect split
+    assert min(loads) >= 8 * 2048 // 74 - 16
+
+
+def test_single_part_never_splits():
+    L = np.arange(0, 5000, 37)
+    sched, ns = schedule.plan(L, 1)
+    assert np.all(np.diff(ns) == 1) and int(sched[5]) == 0
+
+
+def test_validate_rejects_a_broken_plan():
+    L = [300, 500]
+    sched, ns = schedule.plan(L, 4)
+    bad = sched.copy()
+    io = schedule.items_offset(4)
+    bad[io + 2] += 1  # first item's end page overlaps the next item
+    with pytest.raises(AssertionError):
+        schedule.validate(bad, ns, L, 4)
