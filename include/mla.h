@@ -136,6 +136,37 @@ mla_status_t mla_last_device_status(const void* workspace, void* stream);
 /* Enqueues a reset of the workspace status word to MLA_OK on `stream`. */
 mla_status_t mla_clear_device_status(void* workspace, void* stream);
 
+/*
+ * Allocation-free decode.  The pages have no counterpart of this call: it is a
+ * deployment aid of this library for callers that cannot allocate device
+ * memory or pass a workspace, e.g. code running during CUDA graph capture,
+ * engine plugins whose enqueue step may not allocate, or servers that have
+ * already reserved all device memory for their own pool.
+ *
+ * Same arguments and results as mla_decode_fwd without the workspace: the
+ * split-KV scratch (status word + partial results) lives in a static array
+ * of MLA_NOALLOC_SCRATCH_BYTES inside the library, reserved on every GPU that
+ * loads the library until the process exits.  The call allocates nothing.
+ *   - Returns MLA_ERR_WORKSPACE, enqueuing nothing, when the shape needs more
+ *     scratch than that, i.e. mla_workspace_size(batch, s_q, h_q,
+ *     num_sm_parts) > MLA_NOALLOC_SCRATCH_BYTES (64 MiB: for 128 query rows
+ *     per request, batch + num_sm_parts <= 255).
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents;
+ *     each call resets the status word on `stream` first.  Calls that can
+ *     overlap on the GPU (other streams or host threads) race on the array.
+ * Device-detected errors are recorded in the shared array and are not
+ * reported by this call.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+mla_status_t mla_decode_fwd_noalloc(const void* q, const void* kv_cache, mla_kv_format_t fmt,
+                                    int64_t num_blocks, const int32_t* block_table, int max_pages,
+                                    const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                                    float softmax_scale, int causal, const int32_t* sched,
+                                    const int32_t* num_splits, int num_sm_parts, void* out,
+                                    float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

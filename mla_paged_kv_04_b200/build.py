@@ -7,7 +7,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SOURCES = ["api.cu", "decode.cu", "metadata.cu", "combine.cu"]
+SOURCES = ["api.cu", "decode.cu", "metadata.cu", "combine.cu", "noalloc.cu"]
 OUT = os.path.join(HERE, "libmla_b200.so")
 
 
