@@ -19,8 +19,8 @@ int metadata_max_batch();
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream);
 cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
                                int num_parts, cudaStream_t stream);
-cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_tail, const DecodeParams& p,
-                              int num_parts, cudaStream_t stream);
+cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_scale, const CUtensorMap& tm_rope,
+                              const DecodeParams& p, int num_parts, cudaStream_t stream);
 }  // namespace mla
 
 using namespace mla;
@@ -164,7 +164,7 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
   p.timeout_ns = kDefaultTimeoutNs;
 
   const uint64_t rows = static_cast<uint64_t>(num_blocks) * kPage;
-  CUtensorMap tm_a, tm_b;
+  CUtensorMap tm_a, tm_b, tm_c;
   cudaError_t e;
   if (fmt == MLA_KV_BF16) {
     if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_cache, kDqk, rows, kDqk * 2, 64, kPage,
@@ -174,13 +174,15 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
       return MLA_ERR_CUDA;
     e = launch_decode_bf16(tm_a, tm_b, p, num_sm_parts, s);
   } else {
-    // raw bytes: the latent half (256 B) of a token, and its 144-byte tail (scales + RoPE)
+    // raw bytes of a token: a latent half (256 B), the four scales (16 B), a RoPE half (64 B)
     if (!make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 256, kPage,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 144, kPage,
+        !make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 16, kPage,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 64, kPage,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return MLA_ERR_CUDA;
-    e = launch_decode_fp8(tm_a, tm_b, p, num_sm_parts, s);
+    e = launch_decode_fp8(tm_a, tm_b, tm_c, p, num_sm_parts, s);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
 

@@ -1,39 +1,46 @@
 // MLA decode over a paged KV cache on sm_100a.
 //
-// Design (one CTA pair per "part" of the split-KV schedule, persistent over
-// the part's work items):
-//   * The two CTAs of a cluster split the 576 key dims: CTA r owns latent dims
+// One CTA pair (a 2-CTA cluster) per part of the split-KV schedule, persistent
+// over the part's work items (request, page range).
+//
+//   * The pair splits the 576 key dims: CTA r owns latent dims
 //     [256 r, 256 r + 256) and RoPE dims [512 + 32 r, 512 + 32 r + 32).  Each
 //     CTA gathers only its half of every 64-token page (block_table-driven TMA
-//     loads, 36 KB per page half), so KV crosses HBM once.
-//   * Q (this CTA's 288 dims, up to 128 query rows = s_q * h_q) lives in
-//     tensor memory and is the A operand of S_r = Q_r K_r^T, a tcgen05.mma
-//     with M = 128, N = 64 tokens, K = 288, accumulating fp32 in TMEM.
-//   * The pair swaps its partial S through distributed shared memory
-//     (st.async with transaction-count mbarriers) and both add them in the
-//     same order, so both CTAs hold the identical full S and take identical
-//     softmax decisions.
-//   * Online softmax in the log2 domain with a lazy rescale: the reference max
-//     only moves when the row max grows by more than 8 (a factor 256), so O
-//     is rescaled rarely.  P (bf16) is written to tensor memory.
-//   * O_r += P V_r with V_r = this CTA's latent half of the same smem page
-//     (the value is the first 512 dims of the key), M = 128, N = 256, K = 64,
-//     P taken from tensor memory, V as an MN-major operand of the same
-//     128-byte-swizzled tile the QK^T product read as K-major.
-//   * Epilogue: bf16 out and lse for an unsplit request, fp32 partials for a
+//     loads, 36 KB per page half; the FP8 variant loads the raw 656-byte rows
+//     and dequantises its half in shared memory), so KV crosses HBM once.
+//   * Q (this CTA's 288 dims, up to 128 query rows = s_q * h_q) lives in tensor
+//     memory and is the A operand of the partial S_r = Q_r K_r^T: tcgen05.mma,
+//     M = 128, N = 64 tokens, K = 288, fp32 accumulation in tensor memory.
+//   * Softmax exchange, factorised: exp2(x0 + x1 - M0 - M1) = exp2(x0 - M0) *
+//     exp2(x1 - M1) with x_r = log2(e) * softmax_scale * S_r.  Each CTA
+//     exponentiates its own partial logits against a lazy per-row reference
+//     M_r and sends only those factors (fp16) and M_r to the peer through
+//     distributed shared memory; P = (own fp32 factor) * (peer fp16 factor).
+//     That halves the bytes on the CTA-pair link against shipping the fp32
+//     partial S; each CTA normalises its own half of O with its own row sum.
+//   * O_r += P V_r with V_r = this CTA's 256 latent dims of the same page (the
+//     value is the first 512 dims of the key): M = 128, N = 256, K = 64, P read
+//     from tensor memory, V as an MN-major operand of the same 128-byte-
+//     swizzled tile the QK^T product reads as K-major.
+//   * Epilogue: bf16 out + lse for an unsplit request, fp32 partials for a
 //     split one (merged by the combine kernel).
 //
-// Warp roles (256 threads): warp 0 = TMA producer, warp 1 = MMA issuer,
-// warp 2 = tensor-memory allocator, warp 3 idle, warps 4-7 = softmax and
-// epilogue (thread r of the group owns query row r = tensor-memory lane r).
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer, warp 2 tensor-memory
+// allocator, warp 3 idle; warps 4-11 softmax in two warpgroups, warpgroup w
+// owning token columns [32 w, 32 w + 32) of every 64-token tile, thread
+// (w, r) owning query row r (= tensor-memory lane r); FP8 adds warps 12-15
+// for the dequantisation.
 //
-// Every wait on an mbarrier is bounded (params.timeout_ns); a wait that runs
-// out records MLA_ERR_TIMEOUT in the status word, raises a CTA-wide abort
-// flag and the CTA drains its copies and MMAs, frees tensor memory and exits.
+// Issue order of the MMA warp: QK^T(j) then PV(j-2), two tiles ahead, so that
+// S(j+1) is ready when the softmax asks for it while PV(j-1) still runs.
+//
+// Every mbarrier wait is bounded (params.timeout_ns); a wait that runs out
+// records MLA_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains
+// its copies and MMAs, frees tensor memory and exits.
 #include <cuda.h>
-#include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
+#include <cuda_runtime.h>
 #include <math_constants.h>
 
 #include "common.cuh"
@@ -45,17 +52,26 @@ namespace dk {
 constexpr int kChunkBytes = kPage * 128;                 // 64 tokens x 64 dims bf16 (SW128)
 constexpr int kRopeBytes = kPage * 64;                   // 64 tokens x 32 dims bf16 (SW64)
 constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;  // 36864: one page half
-constexpr int kXBytes = kRows * kPage * 4;              // 32768: one partial S tile
 constexpr int kRawLatBytes = kPage * 256;               // FP8: this CTA's 256 latent codes per token
-constexpr int kRawTailBytes = kPage * 144;              // FP8: 4 scales + 64 RoPE bf16 per token
-constexpr int kRawBytes = kRawLatBytes + kRawTailBytes; // 25600
+constexpr int kRawScaleBytes = kPage * 16;              // FP8: the 4 fp32 scales per token
+constexpr int kRawRopeBytes = kPage * 64;               // FP8: this CTA's 32 RoPE bf16 per token
+constexpr int kRawBytes = kRawLatBytes + kRawScaleBytes + kRawRopeBytes;  // 21504
 constexpr int kRawStages = 2;
+// Exchange message per tile: fp16 factors [8 chunks of 8 tokens][128 rows][16 B]
+// + the fp32 reference of every row.
+constexpr int kXERegionBytes = 8 * kRows * 16;          // 16384
+constexpr int kXMsgBytes = kXERegionBytes + kRows * 4;  // 16896
+constexpr int kXBufBytes = kXMsgBytes;
+// Tile j + 4 reuses tile j's buffer; by then the peer has consumed tile j
+// (the peer's message for tile j + 2 is only sent after its consume of j).
+constexpr int kXBuffers = 4;
+constexpr int kSoftmaxWarps = 8;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: the lazy reference moves by more than a factor 256
 
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kStages = kFp8 ? 3 : 4;           // bf16 page-half stages
-  static constexpr int kThreads = kFp8 ? 384 : 256;
-  // barrier indices
+  static constexpr int kStages = kFp8 ? 3 : 4;  // bf16 page-half stages
+  static constexpr int kThreads = kFp8 ? 512 : 384;
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kFull + kStages;
   static constexpr int kSFull = kEmpty + kStages;
@@ -63,21 +79,26 @@ struct Cfg {
   static constexpr int kPFull = kSFree + 1;
   static constexpr int kPvDone = kPFull + 1;
   static constexpr int kQReady = kPvDone + 1;
-  static constexpr int kXFull = kQReady + 1;  // two
-  static constexpr int kDrain = kXFull + 2;
-  static constexpr int kRawFull = kDrain + 1;           // FP8 only
+  static constexpr int kXFull = kQReady + 1;  // kXBuffers of them
+  static constexpr int kDrain = kXFull + kXBuffers;
+  static constexpr int kRawFull = kDrain + 1;  // FP8 only
   static constexpr int kRawEmpty = kRawFull + kRawStages;
   static constexpr int kNumBars = kRawEmpty + kRawStages;
-  static constexpr int kRawOffset = kStages * kStageBytes + 2 * kXBytes;
-  static constexpr int kBarOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
+  static constexpr int kXOffset = kStages * kStageBytes;
+  static constexpr int kRawOffset = kXOffset + kXBuffers * kXBufBytes;
+  static constexpr int kMiscOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
+  // per-row partial maxima of the two softmax warpgroups [tile parity][wg][row]
+  // and their row sums [wg][row] (fp32), then barriers, abort flag, tmem base
+  static constexpr int kRowMaxOffset = kMiscOffset;
+  static constexpr int kRowSumOffset = kRowMaxOffset + 4 * kRows * 4;
+  static constexpr int kBarOffset = kRowSumOffset + 2 * kRows * 4;
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;
 };
 // tensor-memory columns (512 allocated)
-constexpr uint32_t kColO = 0;     // 256 fp32 columns: this CTA's half of O
-constexpr uint32_t kColS = 256;   // 64 fp32 columns: partial S
-constexpr uint32_t kColP = 320;   // 32 columns: P as packed bf16 pairs
-constexpr uint32_t kColQ = 352;   // 144 columns: Q (288 bf16) as packed pairs
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kColO = 0;    // 256 fp32 columns: this CTA's half of O
+constexpr uint32_t kColS = 256;  // 64 fp32 columns: partial S
+constexpr uint32_t kColP = 320;  // 32 columns: P as packed bf16 pairs
+constexpr uint32_t kColQ = 352;  // 144 columns: Q (288 bf16) as packed pairs
 }  // namespace dk
 
 __device__ const int g_never_abort = 0;
@@ -103,6 +124,10 @@ __device__ __forceinline__ void raise_abort(const DecodeParams& p, volatile int*
   *abort_flag = 1;
 }
 
+// Named barrier over the eight softmax warps (id 0 is __syncthreads).
+__device__ __forceinline__ void softmax_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(dk::kSoftmaxWarps * 32) : "memory");
+}
 
 // 16 E4M3 codes (one 16-byte raw unit) times an fp32 scale -> 16 bf16 (RNE),
 // as 8 packed pairs in memory order.  e4m3 -> f16 is exact; the product is
@@ -125,7 +150,7 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float sc, uint32_t (&
 template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                  const DecodeParams p) {
+                  const __grid_constant__ CUtensorMap tm_c, const DecodeParams p) {
   using namespace dk;
   using C = Cfg<kFp8>;
   constexpr int kStages = C::kStages;
@@ -134,9 +159,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw_addr);
   const uint32_t stage0 = base;
-  const uint32_t xbuf0 = base + kStages * kStageBytes;
+  const uint32_t xbuf0 = base + C::kXOffset;
   const uint32_t rawbuf0 = base + C::kRawOffset;
   const uint32_t bar0 = base + C::kBarOffset;
+  float* rowmax_sm = reinterpret_cast<float*>(sbase + C::kRowMaxOffset);
+  float* rowsum_sm = reinterpret_cast<float*>(sbase + C::kRowSumOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::kBarOffset + C::kNumBars * 8);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sbase + C::kBarOffset + C::kNumBars * 8 + 4);
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
@@ -163,12 +190,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       mbar_init(BAR(C::kEmpty + i), 1);
     }
     mbar_init(BAR(C::kSFull), 1);
-    mbar_init(BAR(C::kSFree), 4);
-    mbar_init(BAR(C::kPFull), 4);
+    mbar_init(BAR(C::kSFree), kSoftmaxWarps);
+    mbar_init(BAR(C::kPFull), kSoftmaxWarps);
     mbar_init(BAR(C::kPvDone), 1);
-    mbar_init(BAR(C::kQReady), 4);
-    mbar_init(BAR(C::kXFull), 1);
-    mbar_init(BAR(C::kXFull + 1), 1);
+    mbar_init(BAR(C::kQReady), kSoftmaxWarps);
+    for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
     mbar_init(BAR(C::kDrain), 1);
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
@@ -184,6 +210,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (kFp8) tma_prefetch_desc(&tm_c);
   }
   tc_fence_before();
   __syncthreads();
@@ -226,6 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             mbar_arrive_expect_tx(fb, kRawBytes);
             tma_load_2d(dst, &tm_a, fb, static_cast<int>(rank) * 256, y);
             tma_load_2d(dst + kRawLatBytes, &tm_b, fb, 512, y);
+            tma_load_2d(dst + kRawLatBytes + kRawScaleBytes, &tm_c, fb, 528 + static_cast<int>(rank) * 64, y);
           } else {
             const uint32_t dst = stage0 + st * kStageBytes;
             mbar_arrive_expect_tx(fb, kStageBytes);
@@ -247,6 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
       uint32_t g = 0, nitem = 0;
       bool ok = true;
+      // PV of global tile gg (first of its item: overwrite O).
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
         if (!mbar_wait(BAR(C::kPFull), gg & 1u, abort_flag, p.timeout_ns)) return false;
         tc_fence_after();
@@ -266,6 +295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (!mbar_wait(BAR(C::kQReady), nitem & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         ++nitem;
         tc_fence_after();
+        const uint32_t g0 = g;
         for (int j = 0; j < n; ++j, ++g) {
           const uint32_t st = g % kStages;
           if (!mbar_wait(BAR(C::kFull + st), (g / kStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -279,25 +309,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             mma_ts(tmem + kColS, tmem + kColQ + ks * 8, bd, idesc_qk, ks > 0 ? 1u : 0u);
           }
           tc_commit(BAR(C::kSFull));
-          if (j > 0 && !issue_pv(g - 1, j == 1)) { ok = false; break; }
+          if (j >= 2 && !issue_pv(g - 2, j == 2)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!issue_pv(g - 1, n == 1)) { ok = false; break; }
+        for (uint32_t gg = (n >= 2 ? g - 2 : g0); gg < g; ++gg)
+          if (!issue_pv(gg, gg == g0)) { ok = false; break; }
       }
       if (!ok) raise_abort(p, abort_flag);
       // All issued MMAs complete before tensor memory is released.
       tc_commit(BAR(C::kDrain));
       mbar_wait(BAR(C::kDrain), 0, &g_never_abort, 100000000ull);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 4 + kSoftmaxWarps) {
     // ------------------------------------------------------------------ softmax / epilogue
-    const int wq = warp - 4;
-    const int r = threadIdx.x - 128;  // query row == tensor-memory lane
+    const int wg = (warp - 4) >> 2;     // warpgroup: token columns [32 wg, 32 wg + 32)
+    const int wq = warp & 3;            // tensor-memory lane quarter
+    const int r = wq * 32 + lane;       // query row == tensor-memory lane
+    const int sid = threadIdx.x - 128;  // 0..255 among the softmax threads
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t xpeer = mapa_shared(xbuf0, peer);
     const uint32_t xbar_peer = mapa_shared(BAR(C::kXFull), peer);
-    const float4* xlocal = reinterpret_cast<const float4*>(sbase + kStages * kStageBytes);
-    uint32_t g = 0;
+    const uint8_t* xlocal = sbase + C::kXOffset;
+    const float c_log2 = p.scale_log2;
+    uint32_t g = 0;  // global tile counter (tile being consumed)
     bool ok = true;
     const bool row_ok = r < p.M;
     const int qi = r / p.h_q;
@@ -309,20 +343,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       if (n <= 0) {
         if (row_ok) {
           if (slot >= 0) {
-            if (rank == 0) p.lse_part[static_cast<size_t>(slot) * p.M + r] = -CUDART_INF_F;
+            if (rank == 0 && wg == 0) p.lse_part[static_cast<size_t>(slot) * p.M + r] = -CUDART_INF_F;
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256);
-            for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-            if (rank == 0) p.lse[orow] = -CUDART_INF_F;
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256 + wg * 128);
+            for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+            if (rank == 0 && wg == 0) p.lse[orow] = -CUDART_INF_F;
           }
         }
         continue;
       }
-      // Q -> tensor memory (this CTA's 288 dims as 144 packed bf16 pairs).
+      // Q -> tensor memory (this CTA's 288 dims as 144 packed bf16 pairs);
+      // warpgroup 0 writes columns 0-79, warpgroup 1 columns 80-143.
       {
         const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow * kDqk);
 #pragma unroll 1
-        for (int c16 = 0; c16 < 9; ++c16) {
+        for (int c16 = wg * 5; c16 < (wg == 0 ? 5 : 9); ++c16) {
           uint32_t v[16];
           const int e0 = (c16 < 8) ? static_cast<int>(rank) * 256 + c16 * 32 : 512 + static_cast<int>(rank) * 32;
 #pragma unroll
@@ -341,87 +376,115 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (lane == 0) mbar_arrive(BAR(C::kQReady));
       }
       const int vis = p.causal ? min(L, L - p.s_q + qi + 1) : L;
+      // every row sees at least this many keys: tiles below it need no mask
+      const int vis_all = p.causal ? max(0, L - p.s_q + 1) : L;
       const int last_page = (L - 1) / kPage;
-      float m_ref = -CUDART_INF_F, l = 0.f;
-      for (int j = 0; j < n; ++j, ++g) {
-        const int pg = p0 + j;
-        if (!warp_wait(BAR(C::kSFull), g & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      float m_own = -CUDART_INF_F;   // this CTA's lazy reference of row r (log2 units)
+      float m_comb = -CUDART_INF_F;  // combined reference of the last consumed tile
+      float l = 0.f;                 // this warpgroup's part of the row sum
+
+      // Tile gg (page pg): read this warpgroup's 32 partial logits, agree on
+      // the row's lazy reference with the other warpgroup, exponentiate, send
+      // the fp16 factors (+ reference) to the peer CTA.
+      auto produce = [&](uint32_t gg, int pg, float (&e)[32], float& m_sent) -> bool {
+        if (!warp_wait(BAR(C::kSFull), gg & 1u, abort_flag, p.timeout_ns)) return false;
         tc_fence_after();
-        uint32_t s[64];
-        tmem_ld32(trow + kColS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(trow + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        uint32_t s[32];
+        tmem_ld32(trow + kColS + wg * 32, s);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kSFree));
-        // swap partial S with the peer CTA
-        const uint32_t xb = g & 1u;
-        if (r == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXBytes);
-        {
-          const uint32_t rx = xpeer + xb * kXBytes;
-          const uint32_t rbar = xbar_peer + 8u * xb;
+        const int tok0 = pg * kPage + wg * 32;
+        float tmax = -CUDART_INF_F;
+        if (tok0 + 32 <= vis_all) {
 #pragma unroll
-          for (int c4 = 0; c4 < 16; ++c4)
-            st_async_v4(rx + (c4 * 128 + r) * 16, __uint_as_float(s[4 * c4]), __uint_as_float(s[4 * c4 + 1]),
-                        __uint_as_float(s[4 * c4 + 2]), __uint_as_float(s[4 * c4 + 3]), rbar);
-        }
-        if (!warp_wait<true>(BAR(C::kXFull + xb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-        float x[64];
-        float mt = -CUDART_INF_F;
-        const int tok0 = pg * kPage;
-        const float4* xs = xlocal + xb * (kXBytes / 16);
+          for (int t = 0; t < 32; ++t) {
+            e[t] = __uint_as_float(s[t]) * c_log2;
+            tmax = fmaxf(tmax, e[t]);
+          }
+        } else {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 pv = xs[c4 * 128 + r];
-          const float pe[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int t = 4 * c4 + e;
-            float v = (__uint_as_float(s[t]) + pe[e]) * p.scale_log2;
-            v = (tok0 + t < vis) ? v : -CUDART_INF_F;
-            x[t] = v;
-            mt = fmaxf(mt, v);
+          for (int t = 0; t < 32; ++t) {
+            e[t] = (tok0 + t < vis) ? __uint_as_float(s[t]) * c_log2 : -CUDART_INF_F;
+            tmax = fmaxf(tmax, e[t]);
           }
         }
-        const float m_new = fmaxf(m_ref, mt);
-        const bool need = m_new > m_ref + kRescaleThreshold;
-        const float m_use = need ? m_new : m_ref;
-        const float m_sub = (m_use == -CUDART_INF_F) ? 0.f : m_use;
-        uint32_t pk[32];
+        // Row max over both warpgroups' columns; the buffer alternates with the
+        // tile parity, so one barrier per tile keeps writes and reads apart.
+        float* mx = rowmax_sm + (gg & 1u) * 2 * kRows;
+        mx[wg * kRows + r] = tmax;
+        softmax_bar();
+        tmax = fmaxf(tmax, mx[(wg ^ 1) * kRows + r]);
+        if (tmax > m_own + kRescaleThreshold) m_own = tmax;
+        const float msub = (m_own == -CUDART_INF_F) ? 0.f : m_own;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) e[t] = ex2_approx(e[t] - msub);
+        m_sent = m_own;
+        const uint32_t xb = gg & (kXBuffers - 1);
+        if (sid == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
+        const uint32_t rx = xpeer + xb * kXBufBytes;
+        const uint32_t rbar = xbar_peer + 8u * xb;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          st_async_v4u(rx + ((wg * 4 + c) * 128 + r) * 16, pack_f16x2(e[8 * c + 0], e[8 * c + 1]),
+                       pack_f16x2(e[8 * c + 2], e[8 * c + 3]), pack_f16x2(e[8 * c + 4], e[8 * c + 5]),
+                       pack_f16x2(e[8 * c + 6], e[8 * c + 7]), rbar);
+        if (wg == 0) st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(m_own), rbar);
+        return true;
+      };
+
+      // Tile gg: combine with the peer's factors into P, rescale O when the
+      // combined reference moved, hand P to the PV MMA.
+      auto consume = [&](uint32_t gg, int j, int pg, const float (&e)[32], float m_mine) -> bool {
+        const uint32_t xb = gg & (kXBuffers - 1);
+        if (!warp_wait<true>(BAR(C::kXFull + xb), (gg / kXBuffers) & 1u, abort_flag, p.timeout_ns)) return false;
+        const uint8_t* xs = xlocal + xb * kXBufBytes;
+        const float m_peer = *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
+        const float m_new = m_mine + m_peer;  // -inf while no key has been visible
+        const bool moved = m_new != m_comb;
+        const float factor = moved ? ((m_comb == -CUDART_INF_F) ? 0.f : ex2_approx(m_comb - m_new)) : 1.f;
+        uint32_t pk[16];
         float rowsum = 0.f;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float a = ex2_approx(x[2 * t] - m_sub);
-          const float c = ex2_approx(x[2 * t + 1] - m_sub);
-          pk[t] = pack_bf16x2(a, c);
-          rowsum += a + c;  // fp32 probabilities: the bf16 rounding of P must not reach lse
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(xs + ((wg * 4 + c) * 128 + r) * 16);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 ep = unpack_f16x2(ww[q]);
+            const float a = e[8 * c + 2 * q] * ep.x;
+            const float bq = e[8 * c + 2 * q + 1] * ep.y;
+            rowsum += a + bq;
+            pk[4 * c + q] = pack_bf16x2(a, bq);
+          }
         }
         // The previous tile's PV must be done: P is single-buffered and O may be rescaled.
-        if (g > 0) {
-          if (!warp_wait(BAR(C::kPvDone), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (gg > 0) {
+          if (!warp_wait(BAR(C::kPvDone), (gg - 1) & 1u, abort_flag, p.timeout_ns)) return false;
           tc_fence_after();
         }
-        const float factor = need ? ex2_approx(m_ref - m_use) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
+          for (int cc = 0; cc < 4; ++cc) {
             uint32_t o[32];
-            tmem_ld32(trow + kColO + cc * 32, o);
+            const uint32_t col = kColO + wg * 128 + cc * 32;
+            tmem_ld32(trow + col, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-            tmem_st16(trow + kColO + cc * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-            tmem_st16(trow + kColO + cc * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+            tmem_st16(trow + col, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+            tmem_st16(trow + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
           }
         }
         l = l * factor + rowsum;
-        m_ref = m_use;
+        m_comb = m_new;
         if constexpr (!kFp8) {
           // Slots past the end of the request on its last page may hold NaN/Inf:
           // zero those V rows so that 0 * garbage cannot reach O.  (The FP8
           // dequant warps write zeros there themselves.)
           if (pg == last_page && (L & (kPage - 1))) {
             const int t0 = L & (kPage - 1);
-            uint8_t* stg = sbase + (g % kStages) * kStageBytes;
-            for (int u = r; u < (kPage - t0) * 32; u += 128) {
+            uint8_t* stg = sbase + (gg % kStages) * kStageBytes;
+            for (int u = sid; u < (kPage - t0) * 32; u += kSoftmaxWarps * 32) {
               const int row = t0 + (u >> 5), w = u & 31;
               *reinterpret_cast<uint4*>(stg + (w >> 3) * kChunkBytes + row * 128 + (w & 7) * 16) =
                   make_uint4(0, 0, 0, 0);
@@ -429,26 +492,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             fence_proxy_async_smem();
           }
         }
-        tmem_st16(trow + kColP, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-        tmem_st16(trow + kColP + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+        tmem_st16(trow + kColP + wg * 16, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kPFull));
+        return true;
+      };
+
+      float ea[32], eb[32];
+      float ma = 0.f, mb = 0.f;
+      ok = produce(g, p0, ea, ma);
+#pragma unroll 1
+      for (int j = 0; ok && j < n; j += 2) {
+        if (j + 1 < n && !(ok = produce(g + 1, p0 + j + 1, eb, mb))) break;
+        if (!(ok = consume(g, j, p0 + j, ea, ma))) break;
+        ++g;
+        if (j + 1 >= n) break;
+        if (j + 2 < n && !(ok = produce(g + 1, p0 + j + 2, ea, ma))) break;
+        if (!(ok = consume(g, j + 1, p0 + j + 1, eb, mb))) break;
+        ++g;
       }
       if (!ok) break;
-      // epilogue
+      // epilogue: both warpgroups' row sums, then this warpgroup's 128 columns of O
+      rowsum_sm[wg * kRows + r] = l;
+      softmax_bar();
+      const float lt = l + rowsum_sm[(wg ^ 1) * kRows + r];
+      softmax_bar();
       if (!warp_wait(BAR(C::kPvDone), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse_val = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float lse_val = lt > 0.f ? (m_comb + __log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
 #pragma unroll 1
-      for (int cc = 0; cc < 8; ++cc) {
+      for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        tmem_ld32(trow + kColO + cc * 32, o);
+        const int col = wg * 128 + cc * 32;  // within this CTA's 256 columns
+        tmem_ld32(trow + kColO + col, o);
         if (row_ok) {
           if (slot < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256 + cc * 32);
+            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256 + col);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
@@ -458,7 +540,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             }
           } else {
             float4* dst = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(slot) * p.M + r) * kDv +
-                                                    rank * 256 + cc * 32);
+                                                    rank * 256 + col);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
@@ -466,18 +548,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           }
         }
       }
-      if (row_ok && rank == 0) {
+      if (row_ok && rank == 0 && wg == 0) {
         if (slot < 0) p.lse[orow] = lse_val;
         else p.lse_part[static_cast<size_t>(slot) * p.M + r] = lse_val;
       }
     }
     if (!ok) raise_abort(p, abort_flag);
-  } else if (kFp8 && warp >= 8) {
-    // ------------------------------------------------------------------ FP8 dequant (warps 8-11)
+  } else if (kFp8 && warp >= 4 + kSoftmaxWarps) {
+    // ------------------------------------------------------------------ FP8 dequant (warps 12-15)
     // Raw 656-byte tokens -> this CTA's bf16 page half, in the same swizzled
     // layout the BF16 path gets from TMA.  Thread dt handles 16-code units
     // u = dt + 128 k: token u / 16, codes 16 (u % 16) .. +16 of the CTA's 256.
-    const int dt = threadIdx.x - 256;
+    const int dt = threadIdx.x - 128 - kSoftmaxWarps * 32;
     uint32_t g = 0;
     bool ok = true;
     for (int it = it_begin; it < it_end && ok; ++it) {
@@ -491,7 +573,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             !warp_wait(BAR(C::kEmpty + st), ((g / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         const int valid = (pg == last_page) ? L - pg * kPage : kPage;
         const uint8_t* rlat = sbase + C::kRawOffset + rs * kRawBytes;
-        const uint8_t* rtail = rlat + kRawLatBytes;
+        const uint8_t* rscale = rlat + kRawLatBytes;
+        const uint8_t* rrope = rscale + kRawScaleBytes;
         uint8_t* dst = sbase + st * kStageBytes;
 #pragma unroll 2
         for (int k = 0; k < 8; ++k) {
@@ -500,7 +583,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           uint32_t w[8];
           if (t < valid) {
             const uint4 codes = *reinterpret_cast<const uint4*>(rlat + t * 256 + g16 * 16);
-            const float sc = *reinterpret_cast<const float*>(rtail + t * 144 + 4 * (2 * static_cast<int>(rank) + (g16 >> 3)));
+            const float sc = *reinterpret_cast<const float*>(rscale + t * 16 + 4 * (2 * static_cast<int>(rank) + (g16 >> 3)));
             dequant16(codes, sc, w);
           } else {
 #pragma unroll
@@ -516,7 +599,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           const int u = dt + 128 * k;
           const int t = u >> 2, w4 = u & 3;
           uint4 v = make_uint4(0, 0, 0, 0);
-          if (t < valid) v = *reinterpret_cast<const uint4*>(rtail + t * 144 + 16 + static_cast<int>(rank) * 64 + w4 * 16);
+          if (t < valid) v = *reinterpret_cast<const uint4*>(rrope + t * 64 + w4 * 16);
           *reinterpret_cast<uint4*>(dst + 4 * kChunkBytes + t * 64 + ((w4 ^ ((t >> 1) & 3)) << 4)) = v;
         }
         fence_proxy_async_smem();
@@ -541,8 +624,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 }
 
 template <bool kFp8>
-static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const DecodeParams& p,
-                                 int num_parts, cudaStream_t stream) {
+static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_c,
+                                 const DecodeParams& p, int num_parts, cudaStream_t stream) {
   using C = dk::Cfg<kFp8>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -551,18 +634,18 @@ static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  decode_kernel<kFp8><<<2 * num_parts, C::kThreads, C::kSmemBytes, stream>>>(tm_a, tm_b, p);
+  decode_kernel<kFp8><<<2 * num_parts, C::kThreads, C::kSmemBytes, stream>>>(tm_a, tm_b, tm_c, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
                                int num_parts, cudaStream_t stream) {
-  return launch_decode<false>(tm_lat, tm_rope, p, num_parts, stream);
+  return launch_decode<false>(tm_lat, tm_rope, tm_rope, p, num_parts, stream);
 }
 
-cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_tail, const DecodeParams& p,
-                              int num_parts, cudaStream_t stream) {
-  return launch_decode<true>(tm_lat, tm_tail, p, num_parts, stream);
+cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_scale, const CUtensorMap& tm_rope,
+                              const DecodeParams& p, int num_parts, cudaStream_t stream) {
+  return launch_decode<true>(tm_lat, tm_scale, tm_rope, p, num_parts, stream);
 }
 
 }  // namespace mla
