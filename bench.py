@@ -69,6 +69,31 @@ def algorithmic_work(w: W.Workload, seqlens: np.ndarray):
     return dict(bytes=kv + q + out + lse + meta, kv_bytes=kv, flops=flops)
 
 
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("decode.cu", "sm100.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "mla_paged_kv_04_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + write) of one decode launch from the committed ncu
+    record, or None if there is none for this workload or the kernel source
+    changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[0] == workload and parts[1] == sha:
+                return int(parts[2]) + int(parts[3])
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -341,10 +366,7 @@ def run_cuda(args, world, rank, local):
     roof.update({"kernel": "decode (+ split-KV combine) via mla_decode_fwd", "peak_source": peaks["source"],
                  "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
                  "avg_ms": dec_avg})
-    traffic_file = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
-    if os.path.exists(traffic_file):
-        with open(traffic_file) as f:
-            roof["traffic"] = json.load(f).get("dram_bytes_per_launch")
+    roof["traffic"] = recorded_traffic(w.name)
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

@@ -25,14 +25,15 @@
 //   * Epilogue: bf16 out + lse for an unsplit request, fp32 partials for a
 //     split one (merged by the combine kernel).
 //
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer, warp 2 tensor-memory
-// allocator, warp 3 idle; warps 4-11 softmax in two warpgroups, warpgroup w
-// owning token columns [32 w, 32 w + 32) of every 64-token tile, thread
-// (w, r) owning query row r (= tensor-memory lane r); FP8 adds warps 12-15
-// for the dequantisation.
-//
-// Issue order of the MMA warp: QK^T(j) then PV(j-2), two tiles ahead, so that
-// S(j+1) is ready when the softmax asks for it while PV(j-1) still runs.
+// Warp roles: warp 0 TMA producer, warp 1 QK^T issuer, warp 2 tensor-memory
+// allocator, warp 3 PV issuer; warps 4-11 softmax in two warpgroups,
+// warpgroup w owning token columns [32 w, 32 w + 32) of every 64-token tile,
+// thread (w, r) owning query row r (= tensor-memory lane r); FP8 adds warps
+// 12-15 for the dequantisation.  tcgen05.mma issue blocks for about the
+// instruction's run time, so QK^T and PV get one issuing thread each: QK^T(j)
+// goes out as soon as S is free and the page has landed, PV(j) as soon as
+// P(j) is written, neither waiting behind the other.  P is double-buffered in
+// tensor memory, so the softmax never waits for PV(j-1) to write P(j).
 //
 // Every mbarrier wait is bounded (params.timeout_ns); a wait that runs out
 // records MLA_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains
@@ -76,29 +77,32 @@ struct Cfg {
   static constexpr int kEmpty = kFull + kStages;
   static constexpr int kSFull = kEmpty + kStages;
   static constexpr int kSFree = kSFull + 1;
-  static constexpr int kPFull = kSFree + 1;
-  static constexpr int kPvDone = kPFull + 1;
-  static constexpr int kQReady = kPvDone + 1;
+  static constexpr int kPFull = kSFree + 1;    // two: one per P buffer
+  static constexpr int kPvDone = kPFull + 2;   // two: one per P buffer
+  static constexpr int kQReady = kPvDone + 2;
   static constexpr int kXFull = kQReady + 1;  // kXBuffers of them
-  static constexpr int kDrain = kXFull + kXBuffers;
-  static constexpr int kRawFull = kDrain + 1;  // FP8 only
+  static constexpr int kDrain = kXFull + kXBuffers;  // two: QK^T and PV issuers
+  static constexpr int kRawFull = kDrain + 2;  // FP8 only
   static constexpr int kRawEmpty = kRawFull + kRawStages;
   static constexpr int kNumBars = kRawEmpty + kRawStages;
   static constexpr int kXOffset = kStages * kStageBytes;
   static constexpr int kRawOffset = kXOffset + kXBuffers * kXBufBytes;
-  static constexpr int kMiscOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
-  // per-row partial maxima of the two softmax warpgroups [tile parity][wg][row]
-  // and their row sums [wg][row] (fp32), then barriers, abort flag, tmem base
-  static constexpr int kRowMaxOffset = kMiscOffset;
-  static constexpr int kRowSumOffset = kRowMaxOffset + 4 * kRows * 4;
+  // Q's RoPE half-slice (128 rows x 32 dims bf16, SW64 K-major) is an SS operand
+  static constexpr int kQRopeOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
+  // per-row partial maxima / row sums of the two softmax warpgroups [wg][row]
+  // (fp32), then barriers, abort flag, tmem base
+  static constexpr int kRowMaxOffset = kQRopeOffset + kRows * 64;
+  static constexpr int kRowSumOffset = kRowMaxOffset + 2 * kRows * 4;
   static constexpr int kBarOffset = kRowSumOffset + 2 * kRows * 4;
-  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;
+  // The dynamic shared memory base is 1024-byte aligned (the driver reserves
+  // the first 1 KB of the window); the kernel checks it at entry.
+  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16;
 };
 // tensor-memory columns (512 allocated)
 constexpr uint32_t kColO = 0;    // 256 fp32 columns: this CTA's half of O
 constexpr uint32_t kColS = 256;  // 64 fp32 columns: partial S
-constexpr uint32_t kColP = 320;  // 32 columns: P as packed bf16 pairs
-constexpr uint32_t kColQ = 352;  // 144 columns: Q (288 bf16) as packed pairs
+constexpr uint32_t kColP = 320;  // 2 x 32 columns: P (packed bf16 pairs), double-buffered
+constexpr uint32_t kColQ = 384;  // 128 columns: Q's 256 latent dims as packed bf16 pairs
 }  // namespace dk
 
 __device__ const int g_never_abort = 0;
@@ -156,7 +160,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  if (raw_addr & 1023u) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
+    return;
+  }
+  const uint32_t base = raw_addr;
   uint8_t* sbase = smem_raw + (base - raw_addr);
   const uint32_t stage0 = base;
   const uint32_t xbuf0 = base + C::kXOffset;
@@ -191,11 +199,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
     mbar_init(BAR(C::kSFull), 1);
     mbar_init(BAR(C::kSFree), kSoftmaxWarps);
-    mbar_init(BAR(C::kPFull), kSoftmaxWarps);
-    mbar_init(BAR(C::kPvDone), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(C::kPFull + i), kSoftmaxWarps);
+      mbar_init(BAR(C::kPvDone + i), 1);
+      mbar_init(BAR(C::kDrain + i), 1);
+    }
     mbar_init(BAR(C::kQReady), kSoftmaxWarps);
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
-    mbar_init(BAR(C::kDrain), 1);
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), 4);
@@ -269,33 +279,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         mbar_wait(BAR(full0 + k % nst), (k / nst) & 1u, &g_never_abort, 100000000ull);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ QK^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
+      const uint32_t qrope = base + C::kQRopeOffset;
       uint32_t g = 0, nitem = 0;
       bool ok = true;
-      // PV of global tile gg (first of its item: overwrite O).
-      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-        if (!mbar_wait(BAR(C::kPFull), gg & 1u, abort_flag, p.timeout_ns)) return false;
-        tc_fence_after();
-        const uint32_t sb = stage0 + (gg % kStages) * kStageBytes;
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t bd = sdesc(sb + ks * 2048, 8192, 1024, kSwizzle128);
-          mma_ts(tmem + kColO, tmem + kColP + ks * 8, bd, idesc_pv, (first && ks == 0) ? 0u : 1u);
-        }
-        tc_commit(BAR(C::kPvDone));
-        tc_commit(BAR(C::kEmpty + gg % kStages));
-        return true;
-      };
       for (int it = it_begin; it < it_end && ok; ++it) {
         const int n = items[4 * it + 2] - items[4 * it + 1];
         if (n <= 0) continue;
         if (!mbar_wait(BAR(C::kQReady), nitem & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         ++nitem;
-        tc_fence_after();
-        const uint32_t g0 = g;
         for (int j = 0; j < n; ++j, ++g) {
           const uint32_t st = g % kStages;
           if (!mbar_wait(BAR(C::kFull + st), (g / kStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -303,22 +297,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           tc_fence_after();
           const uint32_t sb = stage0 + st * kStageBytes;
 #pragma unroll
-          for (int ks = 0; ks < 18; ++ks) {
-            const uint64_t bd = ks < 16 ? sdesc(sb + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024, kSwizzle128)
-                                        : sdesc(sb + 4 * kChunkBytes + (ks - 16) * 32, 16, 512, kSwizzle64);
-            mma_ts(tmem + kColS, tmem + kColQ + ks * 8, bd, idesc_qk, ks > 0 ? 1u : 0u);
-          }
+          for (int ks = 0; ks < 16; ++ks)
+            mma_ts(tmem + kColS, tmem + kColQ + ks * 8,
+                   sdesc(sb + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024, kSwizzle128), idesc_qk,
+                   ks > 0 ? 1u : 0u);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            mma_ss(tmem + kColS, sdesc(qrope + ks * 32, 16, 512, kSwizzle64),
+                   sdesc(sb + 4 * kChunkBytes + ks * 32, 16, 512, kSwizzle64), idesc_qk, 1u);
           tc_commit(BAR(C::kSFull));
-          if (j >= 2 && !issue_pv(g - 2, j == 2)) { ok = false; break; }
         }
-        if (!ok) break;
-        for (uint32_t gg = (n >= 2 ? g - 2 : g0); gg < g; ++gg)
-          if (!issue_pv(gg, gg == g0)) { ok = false; break; }
       }
       if (!ok) raise_abort(p, abort_flag);
       // All issued MMAs complete before tensor memory is released.
       tc_commit(BAR(C::kDrain));
       mbar_wait(BAR(C::kDrain), 0, &g_never_abort, 100000000ull);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
+      uint32_t g = 0;
+      bool ok = true;
+      for (int it = it_begin; it < it_end && ok; ++it) {
+        const int n = items[4 * it + 2] - items[4 * it + 1];
+        for (int j = 0; j < n; ++j, ++g) {
+          const uint32_t pb = g & 1u;
+          if (!mbar_wait(BAR(C::kPFull + pb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sb = stage0 + (g % kStages) * kStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tmem + kColO, tmem + kColP + pb * 32 + ks * 8, sdesc(sb + ks * 2048, 8192, 1024, kSwizzle128),
+                   idesc_pv, (j == 0 && ks == 0) ? 0u : 1u);
+          tc_commit(BAR(C::kPvDone + pb));
+          tc_commit(BAR(C::kEmpty + g % kStages));
+        }
+      }
+      if (!ok) raise_abort(p, abort_flag);
+      tc_commit(BAR(C::kDrain + 1));
+      mbar_wait(BAR(C::kDrain + 1), 0, &g_never_abort, 100000000ull);
     }
   } else if (warp >= 4 && warp < 4 + kSoftmaxWarps) {
     // ------------------------------------------------------------------ softmax / epilogue
@@ -352,14 +370,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         }
         continue;
       }
-      // Q -> tensor memory (this CTA's 288 dims as 144 packed bf16 pairs);
-      // warpgroup 0 writes columns 0-79, warpgroup 1 columns 80-143.
+      // Q -> tensor memory: this CTA's 256 latent dims as 128 packed bf16
+      // pairs (warpgroup w writes columns [64 w, 64 w + 64)); the 32 RoPE dims
+      // go to shared memory (SW64 K-major rows of 64 bytes), warpgroup 1.
       {
         const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow * kDqk);
 #pragma unroll 1
-        for (int c16 = wg * 5; c16 < (wg == 0 ? 5 : 9); ++c16) {
+        for (int c16 = wg * 4; c16 < wg * 4 + 4; ++c16) {
           uint32_t v[16];
-          const int e0 = (c16 < 8) ? static_cast<int>(rank) * 256 + c16 * 32 : 512 + static_cast<int>(rank) * 32;
+          const int e0 = static_cast<int>(rank) * 256 + c16 * 32;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint4 w = row_ok ? __ldg(qrow + e0 / 8 + u) : make_uint4(0, 0, 0, 0);
@@ -369,6 +388,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             v[4 * u + 3] = w.w;
           }
           tmem_st16(trow + kColQ + c16 * 16, v);
+        }
+        if (wg == 1) {
+          uint8_t* qr = sbase + C::kQRopeOffset + r * 64;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 w = row_ok ? __ldg(qrow + (512 + static_cast<int>(rank) * 32) / 8 + u) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(qr + ((u ^ ((r >> 1) & 3)) << 4)) = w;
+          }
+          fence_proxy_async_smem();
         }
         tmem_st_wait();
         tc_fence_before();
@@ -395,26 +423,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kSFree));
         const int tok0 = pg * kPage + wg * 32;
-        float tmax = -CUDART_INF_F;
+        float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
         if (tok0 + 32 <= vis_all) {
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             e[t] = __uint_as_float(s[t]) * c_log2;
-            tmax = fmaxf(tmax, e[t]);
+            mx4[t & 3] = fmaxf(mx4[t & 3], e[t]);
           }
         } else {
 #pragma unroll
           for (int t = 0; t < 32; ++t) {
             e[t] = (tok0 + t < vis) ? __uint_as_float(s[t]) * c_log2 : -CUDART_INF_F;
-            tmax = fmaxf(tmax, e[t]);
+            mx4[t & 3] = fmaxf(mx4[t & 3], e[t]);
           }
         }
-        // Row max over both warpgroups' columns; the buffer alternates with the
-        // tile parity, so one barrier per tile keeps writes and reads apart.
-        float* mx = rowmax_sm + (gg & 1u) * 2 * kRows;
-        mx[wg * kRows + r] = tmax;
+        float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        // row max over both warpgroups' columns
+        rowmax_sm[wg * kRows + r] = tmax;
         softmax_bar();
-        tmax = fmaxf(tmax, mx[(wg ^ 1) * kRows + r]);
+        tmax = fmaxf(tmax, rowmax_sm[(wg ^ 1) * kRows + r]);
+        softmax_bar();
         if (tmax > m_own + kRescaleThreshold) m_own = tmax;
         const float msub = (m_own == -CUDART_INF_F) ? 0.f : m_own;
 #pragma unroll
@@ -444,7 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const bool moved = m_new != m_comb;
         const float factor = moved ? ((m_comb == -CUDART_INF_F) ? 0.f : ex2_approx(m_comb - m_new)) : 1.f;
         uint32_t pk[16];
-        float rowsum = 0.f;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint4 w = *reinterpret_cast<const uint4*>(xs + ((wg * 4 + c) * 128 + r) * 16);
@@ -454,16 +482,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             const float2 ep = unpack_f16x2(ww[q]);
             const float a = e[8 * c + 2 * q] * ep.x;
             const float bq = e[8 * c + 2 * q + 1] * ep.y;
-            rowsum += a + bq;
+            rs4[q] += a + bq;
             pk[4 * c + q] = pack_bf16x2(a, bq);
           }
         }
-        // The previous tile's PV must be done: P is single-buffered and O may be rescaled.
-        if (gg > 0) {
-          if (!warp_wait(BAR(C::kPvDone), (gg - 1) & 1u, abort_flag, p.timeout_ns)) return false;
+        const float rowsum = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        const uint32_t pb = gg & 1u;
+        // P buffer pb was last read by PV(gg - 2)
+        if (gg >= 2) {
+          if (!warp_wait(BAR(C::kPvDone + pb), ((gg - 2) >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
           tc_fence_after();
         }
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
+          // O must be stable: PV(gg - 1) done
+          if (!warp_wait(BAR(C::kPvDone + (pb ^ 1u)), ((gg - 1) >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
+          tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t o[32];
@@ -492,11 +525,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             fence_proxy_async_smem();
           }
         }
-        tmem_st16(trow + kColP + wg * 16, pk);
+        tmem_st16(trow + kColP + pb * 32 + wg * 16, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(C::kPFull));
+        if (lane == 0) mbar_arrive(BAR(C::kPFull + pb));
         return true;
       };
 
@@ -519,7 +552,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       softmax_bar();
       const float lt = l + rowsum_sm[(wg ^ 1) * kRows + r];
       softmax_bar();
-      if (!warp_wait(BAR(C::kPvDone), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      if (!warp_wait(BAR(C::kPvDone + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, abort_flag, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const float lse_val = lt > 0.f ? (m_comb + __log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
