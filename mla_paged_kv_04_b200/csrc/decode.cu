@@ -26,14 +26,19 @@
 //     split one (merged by the combine kernel).
 //
 // Warp roles: warp 0 TMA producer, warp 1 QK^T issuer, warp 2 tensor-memory
-// allocator, warp 3 PV issuer; warps 4-11 softmax in two warpgroups,
-// warpgroup w owning token columns [32 w, 32 w + 32) of every 64-token tile,
-// thread (w, r) owning query row r (= tensor-memory lane r); FP8 adds warps
-// 12-15 for the dequantisation.  tcgen05.mma issue blocks for about the
-// instruction's run time, so QK^T and PV get one issuing thread each: QK^T(j)
-// goes out as soon as S is free and the page has landed, PV(j) as soon as
-// P(j) is written, neither waiting behind the other.  P is double-buffered in
-// tensor memory, so the softmax never waits for PV(j-1) to write P(j).
+// allocator, warp 3 PV issuer; warps 4-11 softmax in two warpgroups that take
+// alternate tiles (warpgroup w the tiles g with g % 2 == w), thread (w, r)
+// owning query row r (= tensor-memory lane r) and all 64 columns of its
+// warpgroup's tiles; FP8 adds warps 12-15 for the dequantisation.  The
+// ping-pong lets one warpgroup wait for its pair message while the other one
+// exponentiates, and no barrier joins the two warpgroups inside a tile.  The
+// per-row lazy reference and the combined reference of the last consumed tile
+// pass from one warpgroup to the other through two mbarrier-guarded shared
+// slots, so the references form one sequence per row exactly as if one
+// warpgroup did all tiles.  tcgen05.mma issue blocks for about the
+// instruction's run time, so QK^T and PV get one issuing thread each (one
+// thread for both would hold QK^T(j + 1) behind PV(j)), with their
+// shared-memory descriptors precomputed.
 //
 // Every mbarrier wait is bounded (params.timeout_ns); a wait that runs out
 // records MLA_ERR_TIMEOUT, raises a CTA-wide abort flag, and the CTA drains
@@ -75,28 +80,34 @@ struct Cfg {
   static constexpr int kThreads = kFp8 ? 512 : 384;
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kFull + kStages;
-  static constexpr int kSFull = kEmpty + kStages;
-  static constexpr int kSFree = kSFull + 1;
-  static constexpr int kPFull = kSFree + 1;    // two: one per P buffer
+  static constexpr int kSFull = kEmpty + kStages;  // two: by tile parity
+  static constexpr int kSFree = kSFull + 2;
+  static constexpr int kPFull = kSFree + 1;    // two: one per P buffer (= per warpgroup)
   static constexpr int kPvDone = kPFull + 2;   // two: one per P buffer
   static constexpr int kQReady = kPvDone + 2;
   static constexpr int kXFull = kQReady + 1;  // kXBuffers of them
   static constexpr int kDrain = kXFull + kXBuffers;  // two: QK^T and PV issuers
-  static constexpr int kRawFull = kDrain + 2;  // FP8 only
+  static constexpr int kPChain = kDrain + 2;   // reference of tile g published
+  static constexpr int kCChain = kPChain + 1;  // combined reference of tile g published
+  static constexpr int kEpi = kCChain + 1;     // both warpgroups' row sums published
+  static constexpr int kRawFull = kEpi + 1;    // FP8 only
   static constexpr int kRawEmpty = kRawFull + kRawStages;
   static constexpr int kNumBars = kRawEmpty + kRawStages;
   static constexpr int kXOffset = kStages * kStageBytes;
   static constexpr int kRawOffset = kXOffset + kXBuffers * kXBufBytes;
   // Q's RoPE half-slice (128 rows x 32 dims bf16, SW64 K-major) is an SS operand
   static constexpr int kQRopeOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
-  // per-row partial maxima / row sums of the two softmax warpgroups [wg][row]
-  // (fp32), then barriers, abort flag, tmem base
-  static constexpr int kRowMaxOffset = kQRopeOffset + kRows * 64;
-  static constexpr int kRowSumOffset = kRowMaxOffset + 2 * kRows * 4;
-  static constexpr int kBarOffset = kRowSumOffset + 2 * kRows * 4;
+  // [row] fp32: the lazy reference of the last produced tile; the combined
+  // reference of the last consumed tile; [wg][row] the row-sum parts at the
+  // item's final scale.  Then barriers, abort flag, tmem base.
+  static constexpr int kRefSlotOffset = kQRopeOffset + kRows * 64;
+  static constexpr int kCombSlotOffset = kRefSlotOffset + kRows * 4;
+  static constexpr int kEpiOffset = kCombSlotOffset + kRows * 4;
+  static constexpr int kBarOffset = kEpiOffset + 2 * kRows * 4;
   // The dynamic shared memory base is 1024-byte aligned (the driver reserves
   // the first 1 KB of the window); the kernel checks it at entry.
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 // tensor-memory columns (512 allocated)
 constexpr uint32_t kColO = 0;    // 256 fp32 columns: this CTA's half of O
@@ -107,11 +118,14 @@ constexpr uint32_t kColQ = 384;  // 128 columns: Q's 256 latent dims as packed b
 
 __device__ const int g_never_abort = 0;
 
-// Warp-uniform bounded wait: lane 0 polls with the time limit, then every
-// lane performs its own (immediately successful) acquire of the same phase.
+// Warp-uniform bounded wait.  Fast path: every lane tries the phase once (a
+// completed phase, the common case, costs one warp-wide try).  Otherwise lane 0
+// polls with the time limit, then every lane performs its own (immediately
+// successful) acquire of the same phase.
 template <bool kCluster = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit) {
+  if (__all_sync(0xffffffffu, kCluster ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity))) return true;
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait<kCluster>(bar, parity, abort, limit);
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -126,11 +140,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const v
 __device__ __forceinline__ void raise_abort(const DecodeParams& p, volatile int* abort_flag) {
   report_status(p.status, kStatusTimeout);
   *abort_flag = 1;
-}
-
-// Named barrier over the eight softmax warps (id 0 is __syncthreads).
-__device__ __forceinline__ void softmax_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(dk::kSoftmaxWarps * 32) : "memory");
 }
 
 // 16 E4M3 codes (one 16-byte raw unit) times an fp32 scale -> 16 bf16 (RNE),
@@ -170,8 +179,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   const uint32_t xbuf0 = base + C::kXOffset;
   const uint32_t rawbuf0 = base + C::kRawOffset;
   const uint32_t bar0 = base + C::kBarOffset;
-  float* rowmax_sm = reinterpret_cast<float*>(sbase + C::kRowMaxOffset);
-  float* rowsum_sm = reinterpret_cast<float*>(sbase + C::kRowSumOffset);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + C::kBarOffset + C::kNumBars * 8);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sbase + C::kBarOffset + C::kNumBars * 8 + 4);
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
@@ -197,15 +204,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       mbar_init(BAR(C::kFull + i), kFp8 ? 4 : 1);  // FP8: the four dequant warps arrive
       mbar_init(BAR(C::kEmpty + i), 1);
     }
-    mbar_init(BAR(C::kSFull), 1);
-    mbar_init(BAR(C::kSFree), kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(BAR(C::kPFull + i), kSoftmaxWarps);
+      mbar_init(BAR(C::kSFull + i), 1);
+      mbar_init(BAR(C::kPFull + i), 4);  // the four warps of the consuming warpgroup
       mbar_init(BAR(C::kPvDone + i), 1);
       mbar_init(BAR(C::kDrain + i), 1);
     }
+    mbar_init(BAR(C::kSFree), 4);
     mbar_init(BAR(C::kQReady), kSoftmaxWarps);
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
+    mbar_init(BAR(C::kPChain), 128);  // every thread of the producing warpgroup
+    mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
+    mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), 4);
@@ -228,6 +238,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   const uint32_t tmem = *tmem_holder;
   cluster_sync();  // the peer's barriers are initialised before any st.async reaches them
 
+  // Register budget per warpgroup.  FP8 launches 512 threads with 128
+  // registers each (65,536 in all) and moves them to the softmax warpgroups:
+  // 64 + 2 x 176 + 96 = 4 x 128.  The only increase is the softmax
+  // warpgroups' at their start, which the two decreases exactly fund; at the
+  // end every warpgroup decreases to 64 for the short common tail.  (An
+  // increase anywhere else could take registers that a softmax warpgroup
+  // still waits for: setmaxnreg.inc blocks until the pool can pay.)
+  static_assert(64 + 2 * 176 + 96 <= 4 * 128, "register split exceeds the launch budget");
+  if (warp < 4) {
+    if constexpr (kFp8) setmaxnreg_dec<64>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -282,7 +302,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     // ------------------------------------------------------------------ QK^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 64, false, false);
-      const uint32_t qrope = base + C::kQRopeOffset;
+      // The descriptor's address field is (shared address >> 4) in its low
+      // bits, so a byte offset o within the window is added as o >> 4.
+      const uint64_t d_lat = sdesc(stage0, 16, 1024, kSwizzle128);
+      const uint64_t d_rope = sdesc(stage0 + 4 * kChunkBytes, 16, 512, kSwizzle64);
+      const uint64_t d_qrope = sdesc(base + C::kQRopeOffset, 16, 512, kSwizzle64);
       uint32_t g = 0, nitem = 0;
       bool ok = true;
       for (int it = it_begin; it < it_end && ok; ++it) {
@@ -295,17 +319,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           if (!mbar_wait(BAR(C::kFull + st), (g / kStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           if (g > 0 && !mbar_wait(BAR(C::kSFree), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sb = stage0 + st * kStageBytes;
+          const uint64_t so = static_cast<uint64_t>((st * kStageBytes) >> 4);
 #pragma unroll
           for (int ks = 0; ks < 16; ++ks)
-            mma_ts(tmem + kColS, tmem + kColQ + ks * 8,
-                   sdesc(sb + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024, kSwizzle128), idesc_qk,
-                   ks > 0 ? 1u : 0u);
+            mma_ts(tmem + kColS, tmem + kColQ + ks * 8, d_lat + so + (((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4),
+                   idesc_qk, ks > 0 ? 1u : 0u);
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks)
-            mma_ss(tmem + kColS, sdesc(qrope + ks * 32, 16, 512, kSwizzle64),
-                   sdesc(sb + 4 * kChunkBytes + ks * 32, 16, 512, kSwizzle64), idesc_qk, 1u);
-          tc_commit(BAR(C::kSFull));
+          for (int ks = 0; ks < 2; ++ks) mma_ss(tmem + kColS, d_qrope + 2 * ks, d_rope + so + 2 * ks, idesc_qk, 1u);
+          tc_commit(BAR(C::kSFull + (g & 1u)));
         }
       }
       if (!ok) raise_abort(p, abort_flag);
@@ -317,6 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     // ------------------------------------------------------------------ PV issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_bf16(128, 256, false, true);
+      const uint64_t d_v = sdesc(stage0, 8192, 1024, kSwizzle128);
       uint32_t g = 0;
       bool ok = true;
       for (int it = it_begin; it < it_end && ok; ++it) {
@@ -325,11 +347,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           const uint32_t pb = g & 1u;
           if (!mbar_wait(BAR(C::kPFull + pb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sb = stage0 + (g % kStages) * kStageBytes;
+          const uint64_t so = static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_ts(tmem + kColO, tmem + kColP + pb * 32 + ks * 8, sdesc(sb + ks * 2048, 8192, 1024, kSwizzle128),
-                   idesc_pv, (j == 0 && ks == 0) ? 0u : 1u);
+            mma_ts(tmem + kColO, tmem + kColP + pb * 32 + ks * 8, d_v + so + ks * (2048 >> 4), idesc_pv,
+                   (j == 0 && ks == 0) ? 0u : 1u);
           tc_commit(BAR(C::kPvDone + pb));
           tc_commit(BAR(C::kEmpty + g % kStages));
         }
@@ -338,18 +360,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       tc_commit(BAR(C::kDrain + 1));
       mbar_wait(BAR(C::kDrain + 1), 0, &g_never_abort, 100000000ull);
     }
-  } else if (warp >= 4 && warp < 4 + kSoftmaxWarps) {
+  }
+  } else if (warp < 4 + kSoftmaxWarps) {
     // ------------------------------------------------------------------ softmax / epilogue
-    const int wg = (warp - 4) >> 2;     // warpgroup: token columns [32 wg, 32 wg + 32)
-    const int wq = warp & 3;            // tensor-memory lane quarter
-    const int r = wq * 32 + lane;       // query row == tensor-memory lane
-    const int sid = threadIdx.x - 128;  // 0..255 among the softmax threads
+    if constexpr (kFp8) setmaxnreg_inc<176>();
+    const int wg = (warp - 4) >> 2;         // warpgroup: the tiles g with g % 2 == wg
+    const int wq = warp & 3;                // tensor-memory lane quarter
+    const int r = wq * 32 + lane;           // query row == tensor-memory lane
+    const int wt = threadIdx.x - 128 * (1 + wg);  // 0..127 within the warpgroup
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t xpeer = mapa_shared(xbuf0, peer);
     const uint32_t xbar_peer = mapa_shared(BAR(C::kXFull), peer);
     const uint8_t* xlocal = sbase + C::kXOffset;
+    float* ref_slot = reinterpret_cast<float*>(sbase + C::kRefSlotOffset);
+    float* comb_slot = reinterpret_cast<float*>(sbase + C::kCombSlotOffset);
+    float* epi_slot = reinterpret_cast<float*>(sbase + C::kEpiOffset);
     const float c_log2 = p.scale_log2;
-    uint32_t g = 0;  // global tile counter (tile being consumed)
+    const float c_abs = fabsf(c_log2);
+    const bool c_neg = c_log2 < 0.f;
+    uint32_t g = 0;      // tile counter of this CTA (every tile, both warpgroups)
+    uint32_t nitem = 0;  // items with at least one page
     bool ok = true;
     const bool row_ok = r < p.M;
     const int qi = r / p.h_q;
@@ -407,100 +437,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       // every row sees at least this many keys: tiles below it need no mask
       const int vis_all = p.causal ? max(0, L - p.s_q + 1) : L;
       const int last_page = (L - 1) / kPage;
-      float m_own = -CUDART_INF_F;   // this CTA's lazy reference of row r (log2 units)
-      float m_comb = -CUDART_INF_F;  // combined reference of the last consumed tile
-      float l = 0.f;                 // this warpgroup's part of the row sum
+      float l = 0.f;                  // this warpgroup's part of the row sum ...
+      float m_l = -CUDART_INF_F;      // ... at this combined reference (log2 units)
 
-      // Tile gg (page pg): read this warpgroup's 32 partial logits, agree on
-      // the row's lazy reference with the other warpgroup, exponentiate, send
-      // the fp16 factors (+ reference) to the peer CTA.
-      auto produce = [&](uint32_t gg, int pg, float (&e)[32], float& m_sent) -> bool {
-        if (!warp_wait(BAR(C::kSFull), gg & 1u, abort_flag, p.timeout_ns)) return false;
+#pragma unroll 1
+      for (int j = wg ^ static_cast<int>(g & 1u); j < n; j += 2) {
+        const uint32_t gg = g + static_cast<uint32_t>(j);
+        const int pg = p0 + j;
+        // ---------------------------------------------------------------- produce
+        // read the partial logits of tile gg, fix the row's lazy reference,
+        // exponentiate, send the fp16 factors (+ reference) to the peer CTA
+        if (!warp_wait(BAR(C::kSFull + (gg & 1u)), (gg >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        uint32_t s[32];
-        tmem_ld32(trow + kColS + wg * 32, s);
+        uint32_t s[64];
+        tmem_ld64(trow + kColS, s);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kSFree));
-        const int tok0 = pg * kPage + wg * 32;
-        float mx4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-        if (tok0 + 32 <= vis_all) {
+        const int tok0 = pg * kPage;
+        const bool full_tile = tok0 + kPage <= vis_all;
+        float e[64];
+        float tmax;
+        {
+          float a[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+          if (full_tile) {
+            // max of the raw products; the scale's sign decides max or min
+            if (!c_neg) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            e[t] = __uint_as_float(s[t]) * c_log2;
-            mx4[t & 3] = fmaxf(mx4[t & 3], e[t]);
-          }
-        } else {
+              for (int t = 0; t < 32; ++t)
+                a[t & 3] = fmax3(a[t & 3], __uint_as_float(s[2 * t]), __uint_as_float(s[2 * t + 1]));
+            } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            e[t] = (tok0 + t < vis) ? __uint_as_float(s[t]) * c_log2 : -CUDART_INF_F;
-            mx4[t & 3] = fmaxf(mx4[t & 3], e[t]);
+              for (int t = 0; t < 32; ++t)
+                a[t & 3] = fmax3(a[t & 3], -__uint_as_float(s[2 * t]), -__uint_as_float(s[2 * t + 1]));
+            }
+            tmax = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * c_abs;
+          } else {
+#pragma unroll
+            for (int t = 0; t < 64; ++t) e[t] = (tok0 + t < vis) ? __uint_as_float(s[t]) * c_log2 : -CUDART_INF_F;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) a[t & 3] = fmax3(a[t & 3], e[2 * t], e[2 * t + 1]);
+            tmax = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
           }
         }
-        float tmax = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        // row max over both warpgroups' columns
-        rowmax_sm[wg * kRows + r] = tmax;
-        softmax_bar();
-        tmax = fmaxf(tmax, rowmax_sm[(wg ^ 1) * kRows + r]);
-        softmax_bar();
-        if (tmax > m_own + kRescaleThreshold) m_own = tmax;
-        const float msub = (m_own == -CUDART_INF_F) ? 0.f : m_own;
+        // the reference chain: tile gg continues tile gg - 1's reference
+        if (gg > 0 && !warp_wait(BAR(C::kPChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const float prev = j > 0 ? ref_slot[r] : -CUDART_INF_F;
+        const float ref = (tmax > prev + kRescaleThreshold) ? tmax : prev;
+        ref_slot[r] = ref;
+        mbar_arrive(BAR(C::kPChain));
+        const float msub = (ref == -CUDART_INF_F) ? 0.f : ref;
+        if (full_tile) {
 #pragma unroll
-        for (int t = 0; t < 32; ++t) e[t] = ex2_approx(e[t] - msub);
-        m_sent = m_own;
-        const uint32_t xb = gg & (kXBuffers - 1);
-        if (sid == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
-        const uint32_t rx = xpeer + xb * kXBufBytes;
-        const uint32_t rbar = xbar_peer + 8u * xb;
+          for (int t = 0; t < 64; ++t) e[t] = ex2_approx(fmaf(__uint_as_float(s[t]), c_log2, -msub));
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          st_async_v4u(rx + ((wg * 4 + c) * 128 + r) * 16, pack_f16x2(e[8 * c + 0], e[8 * c + 1]),
-                       pack_f16x2(e[8 * c + 2], e[8 * c + 3]), pack_f16x2(e[8 * c + 4], e[8 * c + 5]),
-                       pack_f16x2(e[8 * c + 6], e[8 * c + 7]), rbar);
-        if (wg == 0) st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(m_own), rbar);
-        return true;
-      };
-
-      // Tile gg: combine with the peer's factors into P, rescale O when the
-      // combined reference moved, hand P to the PV MMA.
-      auto consume = [&](uint32_t gg, int j, int pg, const float (&e)[32], float m_mine) -> bool {
+          for (int t = 0; t < 64; ++t) e[t] = ex2_approx(e[t] - msub);
+        }
         const uint32_t xb = gg & (kXBuffers - 1);
-        if (!warp_wait<true>(BAR(C::kXFull + xb), (gg / kXBuffers) & 1u, abort_flag, p.timeout_ns)) return false;
+        if (wt == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
+        {
+          const uint32_t rx = xpeer + xb * kXBufBytes;
+          const uint32_t rbar = xbar_peer + 8u * xb;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_async_v4u(rx + (c * kRows + r) * 16, pack_f16x2(e[8 * c + 0], e[8 * c + 1]),
+                         pack_f16x2(e[8 * c + 2], e[8 * c + 3]), pack_f16x2(e[8 * c + 4], e[8 * c + 5]),
+                         pack_f16x2(e[8 * c + 6], e[8 * c + 7]), rbar);
+          st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(ref), rbar);
+        }
+        // ---------------------------------------------------------------- consume
+        // combine with the peer's factors into P, rescale O when the combined
+        // reference moved, hand P to the PV MMA
+        if (!warp_wait<true>(BAR(C::kXFull + xb), (gg >> 2) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         const uint8_t* xs = xlocal + xb * kXBufBytes;
-        const float m_peer = *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
-        const float m_new = m_mine + m_peer;  // -inf while no key has been visible
-        const bool moved = m_new != m_comb;
-        const float factor = moved ? ((m_comb == -CUDART_INF_F) ? 0.f : ex2_approx(m_comb - m_new)) : 1.f;
-        uint32_t pk[16];
+        const float m_new = ref + *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
+        if (gg > 0 && !warp_wait(BAR(C::kCChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        const float m_prev = j > 0 ? comb_slot[r] : -CUDART_INF_F;
+        comb_slot[r] = m_new;
+        mbar_arrive(BAR(C::kCChain));
+        uint32_t pk[32];
         float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(xs + ((wg * 4 + c) * 128 + r) * 16);
+        for (int c = 0; c < 8; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(xs + (c * kRows + r) * 16);
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 ep = unpack_f16x2(ww[q]);
-            const float a = e[8 * c + 2 * q] * ep.x;
-            const float bq = e[8 * c + 2 * q + 1] * ep.y;
-            rs4[q] += a + bq;
-            pk[4 * c + q] = pack_bf16x2(a, bq);
+            const float a0 = e[8 * c + 2 * q] * ep.x;
+            const float a1 = e[8 * c + 2 * q + 1] * ep.y;
+            rs4[q] += a0 + a1;
+            pk[4 * c + q] = pack_bf16x2(a0, a1);
           }
         }
         const float rowsum = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         const uint32_t pb = gg & 1u;
         // P buffer pb was last read by PV(gg - 2)
         if (gg >= 2) {
-          if (!warp_wait(BAR(C::kPvDone + pb), ((gg - 2) >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
+          if (!warp_wait(BAR(C::kPvDone + pb), ((gg - 2) >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
         }
+        const bool moved = m_new != m_prev;
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
           // O must be stable: PV(gg - 1) done
-          if (!warp_wait(BAR(C::kPvDone + (pb ^ 1u)), ((gg - 1) >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
+          if (!warp_wait(BAR(C::kPvDone + (pb ^ 1u)), ((gg - 1) >> 1) & 1u, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
+          const float factor = moved ? ((m_prev == -CUDART_INF_F) ? 0.f : ex2_approx(m_prev - m_new)) : 1.f;
 #pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < 8; ++cc) {
             uint32_t o[32];
-            const uint32_t col = kColO + wg * 128 + cc * 32;
+            const uint32_t col = kColO + cc * 32;
             tmem_ld32(trow + col, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
@@ -508,8 +558,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             tmem_st16(trow + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
           }
         }
-        l = l * factor + rowsum;
-        m_comb = m_new;
+        if (m_new != m_l) {
+          l = (m_l == -CUDART_INF_F) ? 0.f : l * ex2_approx(m_l - m_new);
+          m_l = m_new;
+        }
+        l += rowsum;
         if constexpr (!kFp8) {
           // Slots past the end of the request on its last page may hold NaN/Inf:
           // zero those V rows so that 0 * garbage cannot reach O.  (The FP8
@@ -517,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           if (pg == last_page && (L & (kPage - 1))) {
             const int t0 = L & (kPage - 1);
             uint8_t* stg = sbase + (gg % kStages) * kStageBytes;
-            for (int u = sid; u < (kPage - t0) * 32; u += kSoftmaxWarps * 32) {
+            for (int u = wt; u < (kPage - t0) * 32; u += 128) {
               const int row = t0 + (u >> 5), w = u & 31;
               *reinterpret_cast<uint4*>(stg + (w >> 3) * kChunkBytes + row * 128 + (w & 7) * 16) =
                   make_uint4(0, 0, 0, 0);
@@ -525,40 +578,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             fence_proxy_async_smem();
           }
         }
-        tmem_st16(trow + kColP + pb * 32 + wg * 16, pk);
+        tmem_st16(trow + kColP + pb * 32, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(trow + kColP + pb * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kPFull + pb));
-        return true;
-      };
-
-      float ea[32], eb[32];
-      float ma = 0.f, mb = 0.f;
-      ok = produce(g, p0, ea, ma);
-#pragma unroll 1
-      for (int j = 0; ok && j < n; j += 2) {
-        if (j + 1 < n && !(ok = produce(g + 1, p0 + j + 1, eb, mb))) break;
-        if (!(ok = consume(g, j, p0 + j, ea, ma))) break;
-        ++g;
-        if (j + 1 >= n) break;
-        if (j + 2 < n && !(ok = produce(g + 1, p0 + j + 2, ea, ma))) break;
-        if (!(ok = consume(g, j + 1, p0 + j + 1, eb, mb))) break;
-        ++g;
       }
       if (!ok) break;
-      // epilogue: both warpgroups' row sums, then this warpgroup's 128 columns of O
-      rowsum_sm[wg * kRows + r] = l;
-      softmax_bar();
-      const float lt = l + rowsum_sm[(wg ^ 1) * kRows + r];
-      softmax_bar();
-      if (!warp_wait(BAR(C::kPvDone + ((g - 1) & 1u)), ((g - 1) >> 1) & 1u, abort_flag, p.timeout_ns)) {
+      // epilogue: both warpgroups' row sums at the combined reference of the
+      // item's last tile, then this warpgroup's 128 columns of O
+      const uint32_t glast = g + static_cast<uint32_t>(n) - 1u;
+      g += static_cast<uint32_t>(n);
+      float m_fin = m_l;  // this warpgroup consumed the last tile
+      if ((glast & 1u) != static_cast<uint32_t>(wg)) {
+        if (!warp_wait(BAR(C::kCChain), glast & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        m_fin = comb_slot[r];
+      }
+      const float lw = (m_l == -CUDART_INF_F) ? 0.f : l * ex2_approx(m_l - m_fin);
+      epi_slot[wg * kRows + r] = lw;
+      mbar_arrive(BAR(C::kEpi));
+      if (!warp_wait(BAR(C::kEpi), nitem & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      ++nitem;
+      const float lt = lw + epi_slot[(wg ^ 1) * kRows + r];
+      if (!warp_wait(BAR(C::kPvDone + (glast & 1u)), (glast >> 1) & 1u, abort_flag, p.timeout_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float lse_val = lt > 0.f ? (m_comb + __log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
+      const float lse_val = lt > 0.f ? (m_fin + __log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
@@ -590,8 +639,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       }
     }
     if (!ok) raise_abort(p, abort_flag);
-  } else if (kFp8 && warp >= 4 + kSoftmaxWarps) {
+    __syncwarp();
+    if constexpr (kFp8) setmaxnreg_dec<64>();
+  } else if (kFp8) {
     // ------------------------------------------------------------------ FP8 dequant (warps 12-15)
+    setmaxnreg_dec<96>();
     // Raw 656-byte tokens -> this CTA's bf16 page half, in the same swizzled
     // layout the BF16 path gets from TMA.  Thread dt handles 16-code units
     // u = dt + 128 k: token u / 16, codes 16 (u % 16) .. +16 of the CTA's 256.
@@ -647,6 +699,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       }
     }
     if (!ok) raise_abort(p, abort_flag);
+    __syncwarp();
+    setmaxnreg_dec<64>();
   }
 
   tc_fence_before();

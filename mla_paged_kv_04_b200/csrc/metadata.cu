@@ -1,5 +1,6 @@
 // Split-KV schedule for variable-length batches, computed on the device by a
-// single 1024-thread block so that it stays on the caller's stream.
+// single block (one thread per request, up to 1024) so that it stays on the
+// caller's stream.
 //
 // Cost model: request b costs n_b + c units, n_b = ceil(L_b / 64) pages and
 // c = kSplitOverheadPages.  The requests' cost intervals are laid end to end
@@ -28,10 +29,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
     int y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
+  const int nwarps = static_cast<int>(blockDim.x) >> 5;
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = (lane < (kMetaThreads / 32)) ? warp_sums[lane] : 0;
+    int w = (lane < nwarps) ? warp_sums[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -41,7 +43,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
   }
   __syncthreads();
   int prefix = x - v + (warp > 0 ? warp_sums[warp - 1] : 0);
-  *total = warp_sums[kMetaThreads / 32 - 1];
+  *total = warp_sums[nwarps - 1];
   __syncthreads();
   return prefix;
 }
@@ -54,7 +56,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
   int* S = sm + batch + 1;     // [batch + 1] split prefix
   __shared__ int warp_sums[32];
 
-  const int per = (batch + kMetaThreads - 1) / kMetaThreads;
+  const int per = (batch + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
   const int b0 = threadIdx.x * per;
   const int b1 = min(batch, b0 + per);
 
@@ -157,8 +159,11 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int parts, int32_
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, parts, kSplitOverheadPages, sched,
-                                                     num_splits);
+  // one request per thread up to 1024 requests (whole warps): small batches
+  // sync fewer warps in the block scans
+  const int threads = batch >= kMetaThreads ? kMetaThreads : ((batch + 31) / 32) * 32;
+  metadata_kernel<<<1, threads > 0 ? threads : 32, smem, stream>>>(seqlens, batch, parts, kSplitOverheadPages,
+                                                                  sched, num_splits);
   return cudaGetLastError();
 }
 
