@@ -62,21 +62,22 @@ constexpr int kRawLatBytes = kPage * 256;               // FP8: this CTA's 256 l
 constexpr int kRawScaleBytes = kPage * 16;              // FP8: the 4 fp32 scales per token
 constexpr int kRawRopeBytes = kPage * 64;               // FP8: this CTA's 32 RoPE bf16 per token
 constexpr int kRawBytes = kRawLatBytes + kRawScaleBytes + kRawRopeBytes;  // 21504
-constexpr int kRawStages = 2;
+constexpr int kRawStages = 3;
 // Exchange message per tile: fp16 factors [8 chunks of 8 tokens][128 rows][16 B]
 // + the fp32 reference of every row.
 constexpr int kXERegionBytes = 8 * kRows * 16;          // 16384
 constexpr int kXMsgBytes = kXERegionBytes + kRows * 4;  // 16896
 constexpr int kXBufBytes = kXMsgBytes;
-// Tile j + 4 reuses tile j's buffer; by then the peer has consumed tile j
-// (the peer's message for tile j + 2 is only sent after its consume of j).
-constexpr int kXBuffers = 4;
+// Two receive buffers, one per softmax warpgroup (tile g uses buffer g % 2).
+// The peer writes tile g + 2's message into buffer g % 2 only after this CTA
+// has read tile g's (a remote arrive on the peer's "buffer free" barrier).
+constexpr int kXBuffers = 2;
 constexpr int kSoftmaxWarps = 8;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: the lazy reference moves by more than a factor 256
 
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kStages = kFp8 ? 3 : 4;  // bf16 page-half stages
+  static constexpr int kStages = kFp8 ? 3 : 5;  // bf16 page-half stages
   static constexpr int kThreads = kFp8 ? 512 : 384;
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kFull + kStages;
@@ -90,7 +91,8 @@ struct Cfg {
   static constexpr int kPChain = kDrain + 2;   // reference of tile g published
   static constexpr int kCChain = kPChain + 1;  // combined reference of tile g published
   static constexpr int kEpi = kCChain + 1;     // both warpgroups' row sums published
-  static constexpr int kRawFull = kEpi + 1;    // FP8 only
+  static constexpr int kXFree = kEpi + 1;      // two: the peer has read this CTA's message in buffer i
+  static constexpr int kRawFull = kXFree + kXBuffers;  // FP8 only
   static constexpr int kRawEmpty = kRawFull + kRawStages;
   static constexpr int kNumBars = kRawEmpty + kRawStages;
   static constexpr int kXOffset = kStages * kStageBytes;
@@ -216,6 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     mbar_init(BAR(C::kPChain), 128);  // every thread of the producing warpgroup
     mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
     mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
+    for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), 4);
@@ -371,6 +374,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     const uint32_t trow = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t xpeer = mapa_shared(xbuf0, peer);
     const uint32_t xbar_peer = mapa_shared(BAR(C::kXFull), peer);
+    const uint32_t xfree_peer = mapa_shared(BAR(C::kXFree), peer);
     const uint8_t* xlocal = sbase + C::kXOffset;
     float* ref_slot = reinterpret_cast<float*>(sbase + C::kRefSlotOffset);
     float* comb_slot = reinterpret_cast<float*>(sbase + C::kCombSlotOffset);
@@ -496,6 +500,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         }
         const uint32_t xb = gg & (kXBuffers - 1);
         if (wt == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
+        // the peer has read tile gg - 2's message out of the same buffer
+        if (gg >= static_cast<uint32_t>(kXBuffers) &&
+            !warp_wait<true>(BAR(C::kXFree + xb), ((gg - kXBuffers) / kXBuffers) & 1u, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
         {
           const uint32_t rx = xpeer + xb * kXBufBytes;
           const uint32_t rbar = xbar_peer + 8u * xb;
@@ -509,7 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         // ---------------------------------------------------------------- consume
         // combine with the peer's factors into P, rescale O when the combined
         // reference moved, hand P to the PV MMA
-        if (!warp_wait<true>(BAR(C::kXFull + xb), (gg >> 2) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!warp_wait<true>(BAR(C::kXFull + xb), (gg / kXBuffers) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         const uint8_t* xs = xlocal + xb * kXBufBytes;
         const float m_new = ref + *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
         if (gg > 0 && !warp_wait(BAR(C::kCChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -532,6 +542,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           }
         }
         const float rowsum = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        // This warp is done with the peer's message: hand the buffer back.
+        // Every value loaded from it has been consumed by the arithmetic
+        // above (in-order issue), so the loads are complete and a relaxed
+        // arrive is enough to keep the peer's next write behind them.
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * xb);
         const uint32_t pb = gg & 1u;
         // P buffer pb was last read by PV(gg - 2)
         if (gg >= 2) {
