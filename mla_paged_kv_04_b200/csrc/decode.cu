@@ -92,7 +92,8 @@ struct Cfg {
   static constexpr int kCChain = kPChain + 1;  // combined reference of tile g published
   static constexpr int kEpi = kCChain + 1;     // both warpgroups' row sums published
   static constexpr int kXFree = kEpi + 1;      // two: the peer has read this CTA's message in buffer i
-  static constexpr int kRawFull = kXFree + kXBuffers;  // FP8 only
+  static constexpr int kSDone = kXFree + kXBuffers;  // four: QK^T(g) complete, ring by g % 4 (PV issuer)
+  static constexpr int kRawFull = kSDone + 4;  // FP8 only
   static constexpr int kRawEmpty = kRawFull + kRawStages;
   static constexpr int kNumBars = kRawEmpty + kRawStages;
   static constexpr int kXOffset = kStages * kStageBytes;
@@ -219,6 +220,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
     mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
+    for (int i = 0; i < 4; ++i) mbar_init(BAR(C::kSDone + i), 1);
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), 4);
@@ -330,6 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) mma_ss(tmem + kColS, d_qrope + 2 * ks, d_rope + so + 2 * ks, idesc_qk, 1u);
           tc_commit(BAR(C::kSFull + (g & 1u)));
+          tc_commit(BAR(C::kSDone + (g & 3u)));
         }
       }
       if (!ok) raise_abort(p, abort_flag);
@@ -348,6 +351,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const int n = items[4 * it + 2] - items[4 * it + 1];
         for (int j = 0; j < n; ++j, ++g) {
           const uint32_t pb = g & 1u;
+          // PV(g) waits until QK^T(g + 1) of the same item has completed, so
+          // that it runs while the softmax picks up S(g + 1) instead of
+          // delaying QK^T(g + 1) itself (S is single-buffered, so QK^T is on
+          // the softmax's critical loop and PV is not).  The ring of four
+          // barriers cannot alias: QK^T(g + 5) needs the softmax to have
+          // consumed tile g + 2, which waits for PV(g).  The last tile of an
+          // item is not held back (QK^T of the next item waits for its Q,
+          // which waits for this item's epilogue, which waits for PV).
+          if (j + 1 < n &&
+              !mbar_wait(BAR(C::kSDone + ((g + 1) & 3u)), ((g + 1) >> 2) & 1u, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
           if (!mbar_wait(BAR(C::kPFull + pb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
@@ -491,13 +507,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         ref_slot[r] = ref;
         mbar_arrive(BAR(C::kPChain));
         const float msub = (ref == -CUDART_INF_F) ? 0.f : ref;
-        if (full_tile) {
-#pragma unroll
-          for (int t = 0; t < 64; ++t) e[t] = ex2_approx(fmaf(__uint_as_float(s[t]), c_log2, -msub));
-        } else {
-#pragma unroll
-          for (int t = 0; t < 64; ++t) e[t] = ex2_approx(e[t] - msub);
-        }
         const uint32_t xb = gg & (kXBuffers - 1);
         if (wt == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
         // the peer has read tile gg - 2's message out of the same buffer
@@ -507,13 +516,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           break;
         }
         {
+          // Exponentiate and send in two halves of 32 tokens: the first half
+          // crosses to the peer while the second is computed.
           const uint32_t rx = xpeer + xb * kXBufBytes;
           const uint32_t rbar = xbar_peer + 8u * xb;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_async_v4u(rx + (c * kRows + r) * 16, pack_f16x2(e[8 * c + 0], e[8 * c + 1]),
-                         pack_f16x2(e[8 * c + 2], e[8 * c + 3]), pack_f16x2(e[8 * c + 4], e[8 * c + 5]),
-                         pack_f16x2(e[8 * c + 6], e[8 * c + 7]), rbar);
+          for (int h = 0; h < 2; ++h) {
+            if (full_tile) {
+#pragma unroll
+              for (int t = 32 * h; t < 32 * h + 32; ++t) e[t] = ex2_approx(fmaf(__uint_as_float(s[t]), c_log2, -msub));
+            } else {
+#pragma unroll
+              for (int t = 32 * h; t < 32 * h + 32; ++t) e[t] = ex2_approx(e[t] - msub);
+            }
+#pragma unroll
+            for (int c = 4 * h; c < 4 * h + 4; ++c)
+              st_async_v4u(rx + (c * kRows + r) * 16, pack_f16x2(e[8 * c + 0], e[8 * c + 1]),
+                           pack_f16x2(e[8 * c + 2], e[8 * c + 3]), pack_f16x2(e[8 * c + 4], e[8 * c + 5]),
+                           pack_f16x2(e[8 * c + 6], e[8 * c + 7]), rbar);
+          }
           st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(ref), rbar);
         }
         // ---------------------------------------------------------------- consume
