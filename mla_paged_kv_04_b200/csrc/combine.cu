@@ -3,6 +3,8 @@
 // Splits with lse_s = -inf (no visible key, or a zero-page split) get no
 // weight and their partial output is not read.  Each lane of a warp owns 16
 // of the 512 output columns of one query row (four 16-byte loads per split).
+// Summation order: the splits in index order per lane, so the result does not
+// depend on timing.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
@@ -10,12 +12,13 @@
 
 namespace mla {
 
-constexpr int kCombineWarps = 8;
-constexpr int kCombineRowsPerBlock = 32;
+constexpr int kCombineWarps = 4;  // one query row per warp
+constexpr int kCombineUnroll = 4;  // splits whose partial rows are in flight at once
 
 // grid.x walks the schedule's list of split requests (at most one per CTA
-// pair), grid.y covers the query rows 32 at a time; eight warps per block,
-// one query row per warp at a time.
+// pair), grid.y covers the query rows four at a time, one row per warp.  Lane
+// s holds split s's weight (in chunks of 32 splits); the partial rows of
+// kCombineUnroll splits are loaded together so that their latencies overlap.
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineParams p) {
   if (p.sched[0] != p.num_parts) return;  // reported by the decode kernel
   const int num_split_req = p.sched[5];
@@ -25,9 +28,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
   const int first = p.num_splits[b];
   const int nsplit = p.num_splits[b + 1] - first;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int rr = warp; rr < kCombineRowsPerBlock; rr += kCombineWarps) {
-  const int r = blockIdx.y * kCombineRowsPerBlock + rr;
-  if (r >= p.M) break;
+  const int r = blockIdx.y * kCombineWarps + warp;
+  if (r >= p.M) return;
 
   float m = -CUDART_INF_F;
   for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, p.lse_part[static_cast<size_t>(first + s) * p.M + r]);
@@ -37,25 +39,44 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float wsum = 0.f;
+  float wsum = 0.f;  // this lane's splits; reduced over the warp below
   if (m != -CUDART_INF_F) {
-    for (int s = 0; s < nsplit; ++s) {
-      const size_t row = static_cast<size_t>(first + s) * p.M + r;
-      const float ls = p.lse_part[row];
-      if (ls == -CUDART_INF_F) continue;
-      const float w = expf(ls - m);
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+      float w = 0.f;
+      if (s0 + lane < nsplit) {
+        const float ls = p.lse_part[static_cast<size_t>(first + s0 + lane) * p.M + r];
+        w = (ls == -CUDART_INF_F) ? 0.f : expf(ls - m);
+      }
       wsum += w;
-      const float4* src = reinterpret_cast<const float4*>(p.o_part + row * kDv) + lane * 4;
+      const int cnt = min(32, nsplit - s0);
+      for (int k = 0; k < cnt; k += kCombineUnroll) {
+        float wk[kCombineUnroll];
+        float4 x[kCombineUnroll][4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        float4 x = src[v];
-        acc[4 * v + 0] += w * x.x;
-        acc[4 * v + 1] += w * x.y;
-        acc[4 * v + 2] += w * x.z;
-        acc[4 * v + 3] += w * x.w;
+        for (int u = 0; u < kCombineUnroll; ++u) {
+          wk[u] = __shfl_sync(0xffffffffu, w, (k + u) & 31);
+          if (k + u >= cnt) wk[u] = 0.f;
+          const float4* src =
+              reinterpret_cast<const float4*>(p.o_part + (static_cast<size_t>(first + s0 + k + u) * p.M + r) * kDv) +
+              lane * 4;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) x[u][v] = wk[u] != 0.f ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kCombineUnroll; ++u) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            acc[4 * v + 0] += wk[u] * x[u][v].x;
+            acc[4 * v + 1] += wk[u] * x[u][v].y;
+            acc[4 * v + 2] += wk[u] * x[u][v].z;
+            acc[4 * v + 3] += wk[u] * x[u][v].w;
+          }
+        }
       }
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   uint32_t packed[8];
 #pragma unroll
@@ -68,11 +89,10 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
   dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
   if (lane == 0) p.lse[static_cast<size_t>(b) * p.M + r] = wsum > 0.f ? m + logf(wsum) : -CUDART_INF_F;
-  }
 }
 
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream) {
-  dim3 grid(parts, (p.M + kCombineRowsPerBlock - 1) / kCombineRowsPerBlock);
+  dim3 grid(parts, (p.M + kCombineWarps - 1) / kCombineWarps);
   combine_kernel<<<grid, 32 * kCombineWarps, 0, stream>>>(p);
   return cudaGetLastError();
 }

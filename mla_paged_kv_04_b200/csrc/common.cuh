@@ -20,10 +20,18 @@ constexpr int kFp8TokenBytes = 656;
 // kernel (2 x 128 rows x 512 x 4 B, about 7 bf16 pages of traffic for a
 // 128-row request); a smaller value splits more eagerly.
 constexpr int kSplitOverheadPages = 4;
+// A schedule that splits requests pays for it outside the page loop: the
+// fp32 partial outputs go to memory and come back in the combine kernel, and
+// a CTA pair that serves two items drains and refills its pipeline in
+// between.  When the batch fits one request per CTA pair, the schedule keeps
+// requests whole unless that makes the longest part longer than the balanced
+// cut by more than this many pages.
+constexpr int kSplitPenaltyPages = 16;
 
 // Schedule buffer (int32) written by the metadata kernel:
 //   [0] num_parts  [1] total_items  [2] units per part  [3] batch
-//   [4] overhead   [5] number of split requests  [6..8) reserved
+//   [4] overhead   [5] number of split requests  [6] 1 if whole requests
+//   (one per part, no split), else 0   [7] reserved
 //   [8, 8 + num_parts + 1)          first item index of each part
 //   then num_parts ints             ids of the split requests (first [5] valid)
 //   then (16-byte aligned) 4 ints per item: request b, first page, end page, slot

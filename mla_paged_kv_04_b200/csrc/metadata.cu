@@ -12,6 +12,10 @@
 // its fixed cost, so virtual position v maps to page clamp(v - c, 0, n_b).
 // A split may therefore hold zero pages; the decode kernel then only writes
 // lse = -inf for it and the combine kernel gives it no weight.
+//
+// Whole-request mode: when batch <= parts and the costliest request is at
+// most kSplitPenaltyPages above t, part b serves request b alone (parts past
+// the batch stay idle) and nothing is split.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -48,6 +52,19 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* 
   return prefix;
 }
 
+__device__ __forceinline__ int block_max(int v, int* warp_sums) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = static_cast<int>(blockDim.x) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) warp_sums[warp] = v;
+  __syncthreads();
+  int m = 0;
+  for (int w = 0; w < nwarps; ++w) m = max(m, warp_sums[w]);
+  __syncthreads();
+  return m;
+}
+
 __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                                 int parts, int overhead, int32_t* __restrict__ sched,
                                                                 int32_t* __restrict__ num_splits) {
@@ -75,7 +92,37 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
   }
   if (threadIdx.x == 0) C[batch] = T;
   __syncthreads();
-  const int t = max(1, (T + parts - 1) / parts);
+  int t = max(1, (T + parts - 1) / parts);
+
+  // whole-request mode?
+  int local_max = 0;
+  for (int b = b0; b < b1; ++b) local_max = max(local_max, C[b + 1] - C[b]);
+  const int max_cost = block_max(local_max, warp_sums);
+  if (batch <= parts && max_cost <= t + kSplitPenaltyPages) {
+    int32_t* part_first = sched + kSchedHeader;
+    int32_t* items = sched + sched_items_offset(parts);
+    for (int b = b0; b < b1; ++b) {
+      const int L = max(seqlens[b], 0);
+      items[4 * b + 0] = b;
+      items[4 * b + 1] = 0;
+      items[4 * b + 2] = (L + kPage - 1) / kPage;
+      items[4 * b + 3] = -1;
+      num_splits[b] = b;
+    }
+    for (int k = threadIdx.x; k <= parts; k += blockDim.x) part_first[k] = min(k, batch);
+    if (threadIdx.x == 0) {
+      num_splits[batch] = batch;
+      sched[0] = parts;
+      sched[1] = batch;
+      sched[2] = max_cost;
+      sched[3] = batch;
+      sched[4] = overhead;
+      sched[5] = 0;
+      sched[6] = 1;
+      sched[7] = 0;
+    }
+    return;
+  }
 
   // 2. splits per request and their prefix
   local = 0;

@@ -8,7 +8,7 @@ per-part work lists.
 
 Buffer layout (int32):
   [0] parts [1] items [2] units per part [3] batch [4] per-request overhead
-  [5] split requests [6..8) reserved
+  [5] split requests [6] 1 in whole-request mode [7] reserved
   [8, 8 + parts + 1)      first item of each part
   then `parts` ints       ids of split requests (first [5] valid)
   then, 16-byte aligned,  4 ints per item: request, first page, end page, slot
@@ -21,6 +21,11 @@ import numpy as np
 PAGE = 64
 HEADER = 8
 DEFAULT_OVERHEAD = 4
+# Whole-request mode (one request per part, nothing split) is taken when the
+# batch fits the parts and the costliest request exceeds the balanced cut by
+# at most this many pages: splitting costs a round trip of fp32 partials, the
+# combine pass and a pipeline drain per extra item.
+SPLIT_PENALTY = 16
 
 
 def split_list_offset(parts: int) -> int:
@@ -44,6 +49,14 @@ def plan(seqlens, parts: int, overhead: int = DEFAULT_OVERHEAD):
     C = np.concatenate([[0], np.cumsum(cost)])
     T = int(C[-1])
     t = max(1, -(-T // parts))
+    if B <= parts and int(cost.max(initial=0)) <= t + SPLIT_PENALTY:
+        sched = np.zeros(sched_ints(B, parts), dtype=np.int32)
+        sched[:8] = (parts, B, int(cost.max(initial=0)), B, overhead, 0, 1, 0)
+        sched[HEADER:HEADER + parts + 1] = np.minimum(np.arange(parts + 1), B)
+        io = items_offset(parts)
+        items = np.stack([np.arange(B), np.zeros(B, dtype=np.int64), n, np.full(B, -1)], axis=1)
+        sched[io:io + 4 * B] = items.reshape(-1)
+        return sched, np.arange(B + 1, dtype=np.int32)
     k0 = C[:-1] // t
     k1 = (C[1:] - 1) // t
     K = k1 - k0 + 1
