@@ -9,6 +9,7 @@
 #include <math_constants.h>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace mla {
 
@@ -20,6 +21,7 @@ constexpr int kCombineUnroll = 4;  // splits whose partial rows are in flight at
 // s holds split s's weight (in chunks of 32 splits); the partial rows of
 // kCombineUnroll splits are loaded together so that their latencies overlap.
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineParams p) {
+  pdl_wait();  // the decode kernel has completed
   if (p.sched[0] != p.num_parts) return;  // reported by the decode kernel
   const int num_split_req = p.sched[5];
   if (static_cast<int>(blockIdx.x) >= num_split_req) return;
@@ -92,9 +94,16 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
 }
 
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream) {
-  dim3 grid(parts, (p.M + kCombineWarps - 1) / kCombineWarps);
-  combine_kernel<<<grid, 32 * kCombineWarps, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(parts, (p.M + kCombineWarps - 1) / kCombineWarps);
+  cfg.blockDim = dim3(32 * kCombineWarps);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps the decode kernel's tail
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 }  // namespace mla

@@ -31,11 +31,12 @@
 // owning query row r (= tensor-memory lane r) and all 64 columns of its
 // warpgroup's tiles; FP8 adds warps 12-15 for the dequantisation.  The
 // ping-pong lets one warpgroup wait for its pair message while the other one
-// exponentiates, and no barrier joins the two warpgroups inside a tile.  The
-// per-row lazy reference and the combined reference of the last consumed tile
-// pass from one warpgroup to the other through two mbarrier-guarded shared
-// slots, so the references form one sequence per row exactly as if one
-// warpgroup did all tiles.  tcgen05.mma issue blocks for about the
+// exponentiates, and no barrier joins the two warpgroups inside a tile.  Each
+// warpgroup raises its lazy reference to the other's latest published one,
+// read without waiting (any reference is correct; the two converge within a
+// tile or two).  The combined reference of the last consumed tile, which is
+// the scale O is at, passes between them through an mbarrier-guarded slot, so
+// O is rescaled exactly when that scale moves.  tcgen05.mma issue blocks for about the
 // instruction's run time, so QK^T and PV get one issuing thread each (one
 // thread for both would hold QK^T(j + 1) behind PV(j)), with their
 // shared-memory descriptors precomputed.
@@ -88,8 +89,7 @@ struct Cfg {
   static constexpr int kQReady = kPvDone + 2;
   static constexpr int kXFull = kQReady + 1;  // kXBuffers of them
   static constexpr int kDrain = kXFull + kXBuffers;  // two: QK^T and PV issuers
-  static constexpr int kPChain = kDrain + 2;   // reference of tile g published
-  static constexpr int kCChain = kPChain + 1;  // combined reference of tile g published
+  static constexpr int kCChain = kDrain + 2;   // combined reference of tile g published
   static constexpr int kEpi = kCChain + 1;     // both warpgroups' row sums published
   static constexpr int kXFree = kEpi + 1;      // two: the peer has read this CTA's message in buffer i
   static constexpr int kSDone = kXFree + kXBuffers;  // four: QK^T(g) complete, ring by g % 4 (PV issuer)
@@ -100,11 +100,11 @@ struct Cfg {
   static constexpr int kRawOffset = kXOffset + kXBuffers * kXBufBytes;
   // Q's RoPE half-slice (128 rows x 32 dims bf16, SW64 K-major) is an SS operand
   static constexpr int kQRopeOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
-  // [row] fp32: the lazy reference of the last produced tile; the combined
-  // reference of the last consumed tile; [wg][row] the row-sum parts at the
-  // item's final scale.  Then barriers, abort flag, tmem base.
+  // [wg][row] fp32: each warpgroup's latest lazy reference; [row] the
+  // combined reference of the last consumed tile; [wg][row] the row-sum parts
+  // at the item's final scale.  Then barriers, abort flag, tmem base.
   static constexpr int kRefSlotOffset = kQRopeOffset + kRows * 64;
-  static constexpr int kCombSlotOffset = kRefSlotOffset + kRows * 4;
+  static constexpr int kCombSlotOffset = kRefSlotOffset + 2 * kRows * 4;
   static constexpr int kEpiOffset = kCombSlotOffset + kRows * 4;
   static constexpr int kBarOffset = kEpiOffset + 2 * kRows * 4;
   // The dynamic shared memory base is 1024-byte aligned (the driver reserves
@@ -171,8 +171,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   using C = Cfg<kFp8>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
+  // The combine kernel may start launching now; it waits for this grid.
+  pdl_launch_dependents();
   const uint32_t raw_addr = smem_u32(smem_raw);
   if (raw_addr & 1023u) {  // swizzled tiles need 1024-byte alignment
+    pdl_wait();
     if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
     return;
   }
@@ -190,17 +193,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int part = static_cast<int>(cluster_id_x());
-  const int num_parts = p.sched[0];
-  const int32_t* items = p.sched + sched_items_offset(num_parts);
-  int it_begin = 0, it_end = 0;
-  if (num_parts != p.num_parts) {
-    // schedule made for another CTA-pair count: its item slots may not fit
-    // the workspace, so do nothing and report it
-    if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
-  } else {
-    it_begin = p.sched[kSchedHeader + part];
-    it_end = p.sched[kSchedHeader + part + 1];
-  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -216,7 +208,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     mbar_init(BAR(C::kSFree), 4);
     mbar_init(BAR(C::kQReady), kSoftmaxWarps);
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
-    mbar_init(BAR(C::kPChain), 128);  // every thread of the producing warpgroup
     mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
     mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
@@ -242,6 +233,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   cluster_sync();  // the peer's barriers are initialised before any st.async reaches them
+
+  // Everything above touched only this CTA's own memories.  The schedule was
+  // written by the previous kernel in the stream (mla_get_metadata), and the
+  // workspace and outputs may still be read by the previous combine pass.
+  pdl_wait();
+  const int num_parts = p.sched[0];
+  const int32_t* items = p.sched + sched_items_offset(num_parts);
+  int it_begin = 0, it_end = 0;
+  if (num_parts != p.num_parts) {
+    // schedule made for another CTA-pair count: its item slots may not fit
+    // the workspace, so do nothing and report it
+    if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
+  } else {
+    it_begin = p.sched[kSchedHeader + part];
+    it_end = p.sched[kSchedHeader + part + 1];
+  }
 
   // Register budget per warpgroup.  FP8 launches 512 threads with 128
   // registers each (65,536 in all) and moves them to the softmax warpgroups:
@@ -392,7 +399,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     const uint32_t xbar_peer = mapa_shared(BAR(C::kXFull), peer);
     const uint32_t xfree_peer = mapa_shared(BAR(C::kXFree), peer);
     const uint8_t* xlocal = sbase + C::kXOffset;
-    float* ref_slot = reinterpret_cast<float*>(sbase + C::kRefSlotOffset);
+    volatile float* ref_slot = reinterpret_cast<volatile float*>(sbase + C::kRefSlotOffset);
+    ref_slot[wg * kRows + r] = -CUDART_INF_F;
     float* comb_slot = reinterpret_cast<float*>(sbase + C::kCombSlotOffset);
     float* epi_slot = reinterpret_cast<float*>(sbase + C::kEpiOffset);
     const float c_log2 = p.scale_log2;
@@ -425,20 +433,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       // go to shared memory (SW64 K-major rows of 64 bytes), warpgroup 1.
       {
         const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow * kDqk);
-#pragma unroll 1
-        for (int c16 = wg * 4; c16 < wg * 4 + 4; ++c16) {
-          uint32_t v[16];
-          const int e0 = static_cast<int>(rank) * 256 + c16 * 32;
+        // all sixteen 16-byte loads first, so their latencies overlap
+        uint32_t v[4][16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int e0 = static_cast<int>(rank) * 256 + (wg * 4 + c) * 32;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint4 w = row_ok ? __ldg(qrow + e0 / 8 + u) : make_uint4(0, 0, 0, 0);
-            v[4 * u + 0] = w.x;
-            v[4 * u + 1] = w.y;
-            v[4 * u + 2] = w.z;
-            v[4 * u + 3] = w.w;
+            v[c][4 * u + 0] = w.x;
+            v[c][4 * u + 1] = w.y;
+            v[c][4 * u + 2] = w.z;
+            v[c][4 * u + 3] = w.w;
           }
-          tmem_st16(trow + kColQ + c16 * 16, v);
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(trow + kColQ + (wg * 4 + c) * 16, v[c]);
         if (wg == 1) {
           uint8_t* qr = sbase + C::kQRopeOffset + r * 64;
 #pragma unroll
@@ -457,6 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       // every row sees at least this many keys: tiles below it need no mask
       const int vis_all = p.causal ? max(0, L - p.s_q + 1) : L;
       const int last_page = (L - 1) / kPage;
+      float ref_own = -CUDART_INF_F;  // this warpgroup's lazy reference of row r
       float l = 0.f;                  // this warpgroup's part of the row sum ...
       float m_l = -CUDART_INF_F;      // ... at this combined reference (log2 units)
 
@@ -500,12 +511,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             tmax = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
           }
         }
-        // the reference chain: tile gg continues tile gg - 1's reference
-        if (gg > 0 && !warp_wait(BAR(C::kPChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-        const float prev = j > 0 ? ref_slot[r] : -CUDART_INF_F;
+        // the reference: this warpgroup's last one, raised to the other
+        // warpgroup's latest (read without waiting; any value works, and the
+        // two converge after a tile or two)
+        const float prev = fmaxf(ref_own, ref_slot[(wg ^ 1) * kRows + r]);
         const float ref = (tmax > prev + kRescaleThreshold) ? tmax : prev;
-        ref_slot[r] = ref;
-        mbar_arrive(BAR(C::kPChain));
+        ref_own = ref;
+        ref_slot[wg * kRows + r] = ref;
         const float msub = (ref == -CUDART_INF_F) ? 0.f : ref;
         const uint32_t xb = gg & (kXBuffers - 1);
         if (wt == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
@@ -634,6 +646,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       }
       const float lw = (m_l == -CUDART_INF_F) ? 0.f : l * ex2_approx(m_l - m_fin);
       epi_slot[wg * kRows + r] = lw;
+      ref_slot[wg * kRows + r] = -CUDART_INF_F;  // the next item starts afresh
       mbar_arrive(BAR(C::kEpi));
       if (!warp_wait(BAR(C::kEpi), nitem & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
       ++nitem;
@@ -761,8 +774,20 @@ static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  decode_kernel<kFp8><<<2 * num_parts, C::kThreads, C::kSmemBytes, stream>>>(tm_a, tm_b, tm_c, p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the CTAs start (barriers, tensor memory)
+  // while the metadata kernel finishes, and wait in the kernel before
+  // reading the schedule.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * num_parts);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<kFp8>, tm_a, tm_b, tm_c, p);
 }
 
 cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,

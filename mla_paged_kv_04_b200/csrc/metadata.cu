@@ -68,6 +68,8 @@ __device__ __forceinline__ int block_max(int v, int* warp_sums) {
 __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                                 int parts, int overhead, int32_t* __restrict__ sched,
                                                                 int32_t* __restrict__ num_splits) {
+  // the decode kernel may begin launching (it waits for this grid to complete)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ int sm[];
   int* C = sm;                 // [batch + 1] cost prefix
   int* S = sm + batch + 1;     // [batch + 1] split prefix

@@ -124,6 +124,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
   }
 }
 
+// Programmatic dependent launch: let the next kernel of the stream begin
+// launching, and wait until the previous kernel has completed with its memory
+// visible.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------
 // TMA (bulk tensor copies, no multicast anywhere in this library)
 // ----------------------------------------------------------------------------
