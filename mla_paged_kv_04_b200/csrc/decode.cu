@@ -87,13 +87,12 @@ struct Cfg {
   static constexpr int kPFull = kSFree + 1;    // two: one per P buffer (= per warpgroup)
   static constexpr int kPvDone = kPFull + 2;   // two: one per P buffer
   static constexpr int kQReady = kPvDone + 2;
-  static constexpr int kXFull = kQReady + 1;  // kXBuffers of them
-  static constexpr int kDrain = kXFull + kXBuffers;  // two: QK^T and PV issuers
+  static constexpr int kXFull = kQReady + 1;  // two per buffer: tokens 0-31, tokens 32-63 + reference
+  static constexpr int kDrain = kXFull + 2 * kXBuffers;  // two: QK^T and PV issuers
   static constexpr int kCChain = kDrain + 2;   // combined reference of tile g published
   static constexpr int kEpi = kCChain + 1;     // both warpgroups' row sums published
   static constexpr int kXFree = kEpi + 1;      // two: the peer has read this CTA's message in buffer i
-  static constexpr int kSDone = kXFree + kXBuffers;  // four: QK^T(g) complete, ring by g % 4 (PV issuer)
-  static constexpr int kRawFull = kSDone + 4;  // FP8 only
+  static constexpr int kRawFull = kXFree + kXBuffers;  // FP8 only
   static constexpr int kRawEmpty = kRawFull + kRawStages;
   static constexpr int kNumBars = kRawEmpty + kRawStages;
   static constexpr int kXOffset = kStages * kStageBytes;
@@ -207,11 +206,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
     mbar_init(BAR(C::kSFree), 4);
     mbar_init(BAR(C::kQReady), kSoftmaxWarps);
-    for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
+    for (int i = 0; i < 2 * kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
     mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
     mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
-    for (int i = 0; i < 4; ++i) mbar_init(BAR(C::kSDone + i), 1);
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), 4);
@@ -339,7 +337,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) mma_ss(tmem + kColS, d_qrope + 2 * ks, d_rope + so + 2 * ks, idesc_qk, 1u);
           tc_commit(BAR(C::kSFull + (g & 1u)));
-          tc_commit(BAR(C::kSDone + (g & 3u)));
         }
       }
       if (!ok) raise_abort(p, abort_flag);
@@ -358,19 +355,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const int n = items[4 * it + 2] - items[4 * it + 1];
         for (int j = 0; j < n; ++j, ++g) {
           const uint32_t pb = g & 1u;
-          // PV(g) waits until QK^T(g + 1) of the same item has completed, so
-          // that it runs while the softmax picks up S(g + 1) instead of
-          // delaying QK^T(g + 1) itself (S is single-buffered, so QK^T is on
-          // the softmax's critical loop and PV is not).  The ring of four
-          // barriers cannot alias: QK^T(g + 5) needs the softmax to have
-          // consumed tile g + 2, which waits for PV(g).  The last tile of an
-          // item is not held back (QK^T of the next item waits for its Q,
-          // which waits for this item's epilogue, which waits for PV).
-          if (j + 1 < n &&
-              !mbar_wait(BAR(C::kSDone + ((g + 1) & 3u)), ((g + 1) >> 2) & 1u, abort_flag, p.timeout_ns)) {
-            ok = false;
-            break;
-          }
           if (!mbar_wait(BAR(C::kPFull + pb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
@@ -520,7 +504,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         ref_slot[wg * kRows + r] = ref;
         const float msub = (ref == -CUDART_INF_F) ? 0.f : ref;
         const uint32_t xb = gg & (kXBuffers - 1);
-        if (wt == 0) mbar_arrive_expect_tx(BAR(C::kXFull + xb), kXMsgBytes);
+        if (wt == 0) {
+          mbar_arrive_expect_tx(BAR(C::kXFull + 2 * xb), kXERegionBytes / 2);
+          mbar_arrive_expect_tx(BAR(C::kXFull + 2 * xb + 1), kXMsgBytes - kXERegionBytes / 2);
+        }
         // the peer has read tile gg - 2's message out of the same buffer
         if (gg >= static_cast<uint32_t>(kXBuffers) &&
             !warp_wait<true>(BAR(C::kXFree + xb), ((gg - kXBuffers) / kXBuffers) & 1u, abort_flag, p.timeout_ns)) {
@@ -531,9 +518,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           // Exponentiate and send in two halves of 32 tokens: the first half
           // crosses to the peer while the second is computed.
           const uint32_t rx = xpeer + xb * kXBufBytes;
-          const uint32_t rbar = xbar_peer + 8u * xb;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
+            const uint32_t rbar = xbar_peer + 8u * (2 * xb + h);
             if (full_tile) {
 #pragma unroll
               for (int t = 32 * h; t < 32 * h + 32; ++t) e[t] = ex2_approx(fmaf(__uint_as_float(s[t]), c_log2, -msub));
@@ -547,33 +534,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
                            pack_f16x2(e[8 * c + 2], e[8 * c + 3]), pack_f16x2(e[8 * c + 4], e[8 * c + 5]),
                            pack_f16x2(e[8 * c + 6], e[8 * c + 7]), rbar);
           }
-          st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(ref), rbar);
+          st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(ref), xbar_peer + 8u * (2 * xb + 1));
         }
         // ---------------------------------------------------------------- consume
         // combine with the peer's factors into P, rescale O when the combined
         // reference moved, hand P to the PV MMA
-        if (!warp_wait<true>(BAR(C::kXFull + xb), (gg / kXBuffers) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        // The two halves of the peer's message complete separately: P of
+        // tokens 0-31 is formed while tokens 32-63 (and the reference, which
+        // P itself does not need) are still crossing.
         const uint8_t* xs = xlocal + xb * kXBufBytes;
+        uint32_t pk[32];
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!warp_wait<true>(BAR(C::kXFull + 2 * xb + h), (gg / kXBuffers) & 1u, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int c = 4 * h; c < 4 * h + 4; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(xs + (c * kRows + r) * 16);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 ep = unpack_f16x2(ww[q]);
+              const float a0 = e[8 * c + 2 * q] * ep.x;
+              const float a1 = e[8 * c + 2 * q + 1] * ep.y;
+              rs4[q] += a0 + a1;
+              pk[4 * c + q] = pack_bf16x2(a0, a1);
+            }
+          }
+        }
+        if (!ok) break;
         const float m_new = ref + *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
         if (gg > 0 && !warp_wait(BAR(C::kCChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         const float m_prev = j > 0 ? comb_slot[r] : -CUDART_INF_F;
         comb_slot[r] = m_new;
         mbar_arrive(BAR(C::kCChain));
-        uint32_t pk[32];
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(xs + (c * kRows + r) * 16);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 ep = unpack_f16x2(ww[q]);
-            const float a0 = e[8 * c + 2 * q] * ep.x;
-            const float a1 = e[8 * c + 2 * q + 1] * ep.y;
-            rs4[q] += a0 + a1;
-            pk[4 * c + q] = pack_bf16x2(a0, a1);
-          }
-        }
         const float rowsum = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
         // This warp is done with the peer's message: hand the buffer back.
         // Every value loaded from it has been consumed by the arithmetic
