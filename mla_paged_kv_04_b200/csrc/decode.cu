@@ -271,6 +271,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       for (int it = it_begin; it < it_end && ok; ++it) {
         const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
+        // This producer runs kStages pages ahead: start this item's Q rows
+        // towards L2 now, so that the softmax warps' Q loads at the item
+        // boundary do not wait on DRAM behind the page stream (rank 0 fetches
+        // whole rows for both CTAs; q rows are contiguous, 1152 B each).
+        if (rank == 0 && p1 > p0) {
+          const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q) + static_cast<size_t>(b) * p.M * (kDqk * 2);
+          const uint32_t bytes = static_cast<uint32_t>(p.M) * (kDqk * 2);
+          for (uint32_t o = 0; o < bytes; o += 16384u) prefetch_l2_bulk(qb + o, min(16384u, bytes - o));
+        }
         for (int pg = p0; pg < p1; ++pg, ++g) {
           const uint32_t st = g % nst;
           if (g >= static_cast<uint32_t>(nst) &&
