@@ -81,6 +81,9 @@ size_t mla_metadata_size(int batch, int num_sm_parts);
  * algorithm, this one is our own).  Every request costs ceil(L/64) pages
  * plus a fixed per-request overhead; the concatenated cost line is cut into
  * num_sm_parts equal pieces, so a request may be split across CTA pairs.
+ * When batch <= num_sm_parts and the costliest request exceeds the balanced
+ * cut by at most 16 pages, every request gets a CTA pair of its own instead
+ * and nothing is split (no partial outputs, no combine work).
  *
  *   cache_seqlens  device int32 [batch], each >= 0
  *   s_q, h_q       query tokens and heads per request (only validated here)
@@ -118,9 +121,12 @@ size_t mla_workspace_size(int batch, int s_q, int h_q, int num_sm_parts);
  *   out            device bf16 [batch, s_q, h_q, 512] (output)
  *   lse            device fp32 [batch, s_q, h_q] (output)
  *   workspace      device buffer of >= mla_workspace_size() bytes
- * Enqueues the decode kernel and, when some request is split, the split-KV
- * combine kernel on `stream`.  Tail slots of a request's last page and blocks
- * it does not reference may hold any bits (NaN/Inf included).
+ * Enqueues the decode kernel and the split-KV combine kernel (whose blocks
+ * exit at once when no request is split) on `stream`.  Both are launched
+ * with programmatic dependent launch: their CTAs may start while the
+ * previous kernel in `stream` is still running, and wait for it to complete
+ * before they read or write any memory.  Tail slots of a request's last page
+ * and blocks it does not reference may hold any bits (NaN/Inf included).
  */
 mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt,
                             int64_t num_blocks, const int32_t* block_table, int max_pages,

@@ -48,3 +48,30 @@ def test_validate_rejects_a_broken_plan():
     bad[io + 2] += 1  # first item's end page overlaps the next item
     with pytest.raises(AssertionError):
         schedule.validate(bad, ns, L, 4)
+
+
+def test_whole_requests_when_the_batch_fits():
+    # 64 equal requests on 74 CTA pairs: one request per pair, nothing split
+    L = [4096] * 64
+    sched, ns = schedule.plan(L, 74)
+    schedule.validate(sched, ns, L, 74)
+    assert int(sched[6]) == 1 and int(sched[5]) == 0
+    assert np.array_equal(np.diff(ns), np.ones(64, dtype=np.int32))
+    parts = schedule.parse(sched, 74)
+    assert [len(x) for x in parts] == [1] * 64 + [0] * 10
+    assert all(parts[b][0] == (b, 0, 64, -1) for b in range(64))
+
+
+def test_imbalanced_batch_is_still_split():
+    # one request far above the balanced cut: splitting wins over the penalty
+    L = [4096] * 63 + [65536]
+    sched, ns = schedule.plan(L, 74)
+    schedule.validate(sched, ns, L, 74)
+    assert int(sched[6]) == 0 and int(sched[5]) >= 1
+
+
+def test_batch_above_parts_uses_the_balanced_cut():
+    L = [4096] * 128
+    sched, ns = schedule.plan(L, 74)
+    schedule.validate(sched, ns, L, 74)
+    assert int(sched[6]) == 0
