@@ -146,7 +146,7 @@ __device__ __forceinline__ void raise_abort(const DecodeParams& p, volatile int*
 
 // 16 E4M3 codes (one 16-byte raw unit) times an fp32 scale -> 16 bf16 (RNE),
 // as 8 packed pairs in memory order.  e4m3 -> f16 is exact; the product is
-// formed in fp32 and rounded once to bf16.
+// formed in fp32 (a packed pair of IEEE multiplies) and rounded once to bf16.
 __device__ __forceinline__ void dequant16(const uint4 raw, float sc, uint32_t (&w)[8]) {
   const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -155,9 +155,9 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float sc, uint32_t (&
     for (int h = 0; h < 2; ++h) {
       const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((in[i] >> (16 * h)) & 0xFFFFu);
       const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      const float lo = __half2float(__ushort_as_half(hr.x));
-      const float hi = __half2float(__ushort_as_half(hr.y));
-      w[2 * i + h] = pack_bf16x2(lo * sc, hi * sc);
+      const float2 v = __fmul2_rn(make_float2(__half2float(__ushort_as_half(hr.x)), __half2float(__ushort_as_half(hr.y))),
+                                  make_float2(sc, sc));
+      w[2 * i + h] = pack_bf16x2(v.x, v.y);
     }
   }
 }
@@ -531,8 +531,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           for (int h = 0; h < 2; ++h) {
             const uint32_t rbar = xbar_peer + 8u * (2 * xb + h);
             if (full_tile) {
+              // the exponent arguments in packed fp32 pairs (one FFMA2 per two)
+              const float2 c2 = make_float2(c_log2, c_log2), nm2 = make_float2(-msub, -msub);
 #pragma unroll
-              for (int t = 32 * h; t < 32 * h + 32; ++t) e[t] = ex2_approx(fmaf(__uint_as_float(s[t]), c_log2, -msub));
+              for (int t = 32 * h; t < 32 * h + 32; t += 2) {
+                const float2 x =
+                    __ffma2_rn(make_float2(__uint_as_float(s[t]), __uint_as_float(s[t + 1])), c2, nm2);
+                e[t] = ex2_approx(x.x);
+                e[t + 1] = ex2_approx(x.y);
+              }
             } else {
 #pragma unroll
               for (int t = 32 * h; t < 32 * h + 32; ++t) e[t] = ex2_approx(e[t] - msub);
@@ -553,7 +560,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         // P itself does not need) are still crossing.
         const uint8_t* xs = xlocal + xb * kXBufBytes;
         uint32_t pk[32];
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // row-sum partials, packed pairs
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (!warp_wait<true>(BAR(C::kXFull + 2 * xb + h), (gg / kXBuffers) & 1u, abort_flag, p.timeout_ns)) {
@@ -566,11 +573,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const float2 ep = unpack_f16x2(ww[q]);
-              const float a0 = e[8 * c + 2 * q] * ep.x;
-              const float a1 = e[8 * c + 2 * q + 1] * ep.y;
-              rs4[q] += a0 + a1;
-              pk[4 * c + q] = pack_bf16x2(a0, a1);
+              const float2 a = __fmul2_rn(make_float2(e[8 * c + 2 * q], e[8 * c + 2 * q + 1]), unpack_f16x2(ww[q]));
+              rs2[q & 1] = __fadd2_rn(rs2[q & 1], a);
+              pk[4 * c + q] = pack_bf16x2(a.x, a.y);
             }
           }
         }
@@ -580,7 +585,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const float m_prev = j > 0 ? comb_slot[r] : -CUDART_INF_F;
         comb_slot[r] = m_new;
         mbar_arrive(BAR(C::kCChain));
-        const float rowsum = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        const float rowsum = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
         // This warp is done with the peer's message: hand the buffer back.
         // Every value loaded from it has been consumed by the arithmetic
         // above (in-order issue), so the loads are complete and a relaxed
