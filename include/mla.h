@@ -125,7 +125,9 @@ size_t mla_workspace_size(int batch, int s_q, int h_q, int num_sm_parts);
  * exit at once when no request is split) on `stream`.  Both are launched
  * with programmatic dependent launch: their CTAs may start while the
  * previous kernel in `stream` is still running, and wait for it to complete
- * before they read or write any memory.  Tail slots of a request's last page
+ * before they read or write any memory.  (Before that wait the decode CTAs
+ * only issue L2 prefetch hints for q and block_table, which read no value.)
+ * Tail slots of a request's last page
  * and blocks it does not reference may hold any bits (NaN/Inf included).
  */
 mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt,

@@ -232,7 +232,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   const uint32_t tmem = *tmem_holder;
   cluster_sync();  // the peer's barriers are initialised before any st.async reaches them
 
-  // Everything above touched only this CTA's own memories.  The schedule was
+  // While the schedule kernel finishes: start q and the block table towards
+  // L2, spread over every thread of the grid, so that the first Q and
+  // block-table reads after the wait do not go to DRAM.  A prefetch only
+  // moves cache lines and cannot observe a value, so it is issued before the
+  // wait whoever writes these tensors.
+  {
+    const size_t nthr = static_cast<size_t>(gridDim.x) * blockDim.x;
+    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const size_t qbytes = static_cast<size_t>(p.batch) * p.M * (kDqk * 2);
+    const size_t btbytes = static_cast<size_t>(p.batch) * p.max_pages * 4;
+    const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q);
+    const uint8_t* btb = reinterpret_cast<const uint8_t*>(p.block_table);
+    for (size_t o = tid * 128; o < qbytes; o += nthr * 128) prefetch_l2_line(qb + o);
+    for (size_t o = tid * 128; o < btbytes; o += nthr * 128) prefetch_l2_line(btb + o);
+  }
+  // Everything above wrote only this CTA's own memories.  The schedule was
   // written by the previous kernel in the stream (mla_get_metadata), and the
   // workspace and outputs may still be read by the previous combine pass.
   pdl_wait();

@@ -120,12 +120,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
       : "memory");
 }
-// Make generic-proxy shared-memory writes visible to the async proxy (TMA,
-// tensor core) before they are consumed there.
+// Prefetch of the cache line holding gptr into L2 (a hint: no completion, no
+// effect on the values later loads see).
+__device__ __forceinline__ void prefetch_l2_line(const void* gptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(gptr) : "memory");
+}
 // Bulk prefetch of global memory into L2 (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* gptr, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");
 }
+// Make generic-proxy shared-memory writes visible to the async proxy (TMA,
+// tensor core) before they are consumed there.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
