@@ -259,3 +259,101 @@ def mla_decode(q_bits: np.ndarray, kv_cache: np.ndarray, fmt: str, block_table: 
 def default_softmax_scale() -> float:
     """576^-0.5, the scale every configured workload uses."""
     return 1.0 / math.sqrt(D_QK)
+
+
+# ---------------------------------------------------------------------------
+# Cache append: writing new tokens into the paged cache
+# ---------------------------------------------------------------------------
+#
+# The pages fix the FP8 token at 656 bytes with the RoPE slice kept in BF16
+# (menfem.com DeepSeek page, "Key Contributions") and name E4M3 (CUTLASS
+# discussion page); how a token is quantised into it is not printed.  Reading
+# R9 (the plainest one the layout R4 supports): per 128-wide latent group g,
+#   scale_g = fp32(amax_g / 448)                (448 = largest finite E4M3)
+#   code_d  = E4M3 round-to-nearest-even of fp32(x_d / scale_g), saturated
+#             to +-448
+# with both divisions IEEE binary32 (correctly rounded); a group with
+# amax_g == 0 gets scale 0 and all codes 0.  The new token's values are finite.
+
+def _e4m3_finite_magnitudes() -> np.ndarray:
+    """Values of the non-negative finite E4M3 codes 0x00..0x7E, ascending."""
+    return decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+
+
+def encode_e4m3_rne(y: np.ndarray) -> np.ndarray:
+    """float32 values -> E4M3 codes (uint8), round to nearest, ties to even.
+
+    Written from the format definition (R5): the result is the finite E4M3
+    value nearest to y; at an exact midpoint between two neighbours the one
+    with an even code (mantissa LSB 0) wins.  Magnitudes beyond 448 saturate
+    to 448.  The sign bit is y's sign bit, so -0.0 and negative values that
+    round to zero give 0x80.  NaN is outside the supported inputs.
+    """
+    v = np.asarray(y, dtype=np.float32).astype(np.float64)
+    mags = _e4m3_finite_magnitudes()  # 127 values, strictly increasing
+    a = np.minimum(np.abs(v), mags[-1])
+    hi = np.clip(np.searchsorted(mags, a, side="left"), 0, mags.size - 1)
+    lo = np.clip(hi - 1, 0, mags.size - 1)
+    d_lo = a - mags[lo]
+    d_hi = mags[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(v), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def quantize_fp8_656(latent_bits: np.ndarray, rope_bits: np.ndarray) -> np.ndarray:
+    """New tokens -> 656-byte FP8 rows (reading R9 above, layout R4).
+
+    latent_bits uint16 [n, 512] and rope_bits uint16 [n, 64] are bf16 bit
+    patterns; the result is uint8 [n, 656]: 512 codes, four little-endian fp32
+    scales, the 64 RoPE bf16 values unchanged.
+    """
+    lat = np.asarray(latent_bits, dtype=np.uint16)
+    n = lat.shape[0]
+    x = decode_bf16_bits(lat).astype(np.float32).reshape(n, FP8_NUM_SCALES, FP8_GROUP)
+    amax = np.abs(x).max(axis=-1)  # exact
+    scale = (amax / np.float32(448.0)).astype(np.float32)  # one IEEE binary32 division
+    codes = np.zeros((n, FP8_NUM_SCALES, FP8_GROUP), dtype=np.uint8)
+    for i in range(n):
+        for g in range(FP8_NUM_SCALES):
+            if scale[i, g] > 0:
+                y = (x[i, g] / scale[i, g]).astype(np.float32)  # IEEE binary32 divisions
+                codes[i, g] = encode_e4m3_rne(y)
+    out = np.empty((n, FP8_TOKEN_BYTES), dtype=np.uint8)
+    out[:, :D_LATENT] = codes.reshape(n, D_LATENT)
+    out[:, D_LATENT:D_LATENT + 16] = np.ascontiguousarray(scale.astype("<f4")).view(np.uint8).reshape(n, 16)
+    out[:, D_LATENT + 16:] = np.ascontiguousarray(np.asarray(rope_bits, dtype="<u2")).view(np.uint8).reshape(n, 128)
+    return out
+
+
+def append_tokens(kv_cache: np.ndarray, fmt: str, new_bits: np.ndarray, block_table: np.ndarray,
+                  cache_seqlens: np.ndarray) -> np.ndarray:
+    """The cache after appending new tokens (returns a modified copy).
+
+    new_bits uint16 [batch, s_new, 576]: bf16 bit patterns of the new keys.
+    cache_seqlens [batch] are the lengths after the append (the ones the next
+    decode call takes), so new token t of request b is token
+    p = L_b - s_new + t of the request and lands in slot p % 64 of physical
+    block block_table[b, p // 64] (R6).  "bf16" stores the bit patterns,
+    "fp8_656" the quantised row (R9).  Rows with p < 0, a page at or beyond
+    the block-table row, or a block index outside the cache are skipped.
+    """
+    out = np.array(kv_cache, copy=True)
+    new = np.asarray(new_bits, dtype=np.uint16)
+    B, s_new, _ = new.shape
+    bt = np.asarray(block_table)
+    num_blocks = out.shape[0]
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        rows = new[b]
+        if fmt == "fp8_656":
+            rows = quantize_fp8_656(rows[:, :D_LATENT], rows[:, D_LATENT:])
+        for t in range(s_new):
+            p = L - s_new + t
+            if p < 0 or p // PAGE_SIZE >= bt.shape[1]:
+                continue
+            blk = int(bt[b, p // PAGE_SIZE])
+            if blk < 0 or blk >= num_blocks:
+                continue
+            out[blk, p % PAGE_SIZE] = rows[t]
+    return out
