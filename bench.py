@@ -7,6 +7,7 @@ flushed (256 MiB write) before every timed step and each step is timed with
 CUDA events on the launching stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py --op append [--workload NAME]   (the cache-append kernel, see run_append)
 
 Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
 replica of the workload (requests are independent, there is no data-path
@@ -446,6 +447,142 @@ def run_cuda(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# the cache-append kernel (mla_kv_append)
+# ---------------------------------------------------------------------------
+
+APPEND_METRIC = "KV-cache append effective HBM GB/s on 1 B200 (frac of roofline)"
+APPEND_TOKENS = 2048  # new tokens per request in the timed append (a chunk of prefill)
+
+
+def append_work(fmt: str, batch: int, s_new: int) -> int:
+    """Algorithmic bytes of one append: the new bf16 rows read, the cache rows
+    written (1,152 or 656 bytes), one block-table entry per token, the lengths."""
+    tokens = batch * s_new
+    return tokens * (1152 + (1152 if fmt == "bf16" else 656)) + 4 * tokens + 4 * batch
+
+
+def oracle_append_rate(w: W.Workload, budget_s: float = 5.0):
+    """The oracle's append on whole-page chunks of new tokens until `budget_s`."""
+    import oracle
+    case = W.make_case(w, seqlens=[256], poison=False)
+    a = W.oracle_arrays(case)
+    g = torch.Generator().manual_seed(7)
+    new = torch.randn((1, 64, 576), generator=g).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        oracle.append_tokens(a["kv_cache"], w.fmt, new, a["block_table"], a["cache_seqlens"])
+        n += 1
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return (append_work(w.fmt, 1, 64) * n / dt / 1e9, f"{n} appends of 64 new tokens into one "
+            f"{w.fmt} request ({dt:.1f} s of oracle time)", cores)
+
+
+def run_append(args, world, rank, local):
+    """Time mla_kv_append: APPEND_TOKENS new tokens into every request of the
+    workload's cache (the last APPEND_TOKENS positions), L2 flushed before each
+    step; also a decode step's append (s_q new tokens per request)."""
+    import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    mla.load_library()
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    case = W.make_case(w, seed=w.seed + rank, device=dev, poison=False)
+    kv, bt, L = case["kv_cache"], case["block_table"], case["cache_seqlens"]
+    B = w.batch
+    s_new = min(APPEND_TOKENS, int(L.min().item()))
+    gen = torch.Generator(device=dev).manual_seed(1000 + rank)
+    new = torch.randn((B, s_new, 576), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    step_new = new[:, -w.s_q:].contiguous()  # a decode step's new tokens
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    work = append_work(w.fmt, B, s_new)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        mla.mla_kv_append(new, kv, w.fmt, bt, L, ws, stream=stream)
+        mla.mla_kv_append(step_new, kv, w.fmt, bt, L, ws, stream=stream)
+    torch.cuda.synchronize(dev)
+    status = mla.mla_last_device_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status {mla.STATUS.get(status, status)} during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index or 0) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            mla.mla_kv_append(new, kv, w.fmt, bt, L, ws, stream=stream)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    small_ms = []
+    for i in range(args.steps):
+        flush.zero_()
+        e1, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e1.record(stream)
+        mla.mla_kv_append(step_new, kv, w.fmt, bt, L, ws, stream=stream)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        small_ms.append(e1.elapsed_time(e2))
+    # end to end through the public call: upload the new tokens from pinned
+    # memory, append, read the status word back
+    new_h = new.cpu().pin_memory()
+    st_h = torch.empty(4, dtype=torch.uint8).pin_memory()
+    new_d = torch.empty_like(new)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for i in range(args.steps):
+        new_d.copy_(new_h, non_blocking=True)
+        mla.mla_kv_append(new_d, kv, w.fmt, bt, L, ws, stream=stream)
+        st_h.copy_(ws[:4], non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), world) / args.steps
+    status = mla.mla_last_device_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status {mla.STATUS.get(status, status)} in the timed region")
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    n = world
+    ms_per_step = total_ms / args.steps
+    achieved = work / (statistics.mean(step_ms) * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, sample, cores = oracle_append_rate(w)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
+    line = {
+        "metric": APPEND_METRIC, "value": n * work / (ms_per_step * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.fmt == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": f"append into {w.describe()}", "op": "append", "batch": B, "s_new": s_new,
+                   "kv_format": w.fmt, "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replicas x{n} (independent request batches)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "append_kernel",
+                     "peak_source": peaks["source"], "algorithmic_bytes": work},
+        "decode_step_append_us": 1000 * statistics.median(small_ms),
+        "cpu_baseline": cpu,
+        "e2e": {"value": n * work / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": new.numel() * 2,
+                "d2h_bytes_per_step": 4, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -456,6 +593,7 @@ def main():
     ap.add_argument("--parts", type=int, default=0, help="CTA pairs (default: SMs / 2)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="decode", choices=["decode", "append"])
     args = ap.parse_args()
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -464,7 +602,7 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_cuda(args, world, rank, local)
+        (run_append if args.op == "append" else run_cuda)(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

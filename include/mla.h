@@ -137,6 +137,42 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
                             const int32_t* num_splits, int num_sm_parts, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Cache append: write new tokens into the paged cache, the step that fills
+ * what mla_decode_fwd reads.  The pages print only the FP8 token's size (656
+ * bytes against 1,152 in BF16, RoPE slice kept in BF16: menfem.com DeepSeek
+ * page, "Key Contributions") and name E4M3 (CUTLASS discussion page); the
+ * quantisation below is this library's reading of that format.
+ *
+ *   kv_new         device bf16 [batch, s_new, 576], row-major, 16-byte aligned:
+ *                  the new tokens' keys (512 latent + 64 RoPE), finite values
+ *   batch, s_new   requests and new tokens per request (>= 1 each)
+ *   cache_seqlens  device int32 [batch]: lengths AFTER the append (the same
+ *                  array the following decode call takes).  New token t of
+ *                  request b is token p = cache_seqlens[b] - s_new + t and is
+ *                  written to slot p % 64 of block block_table[b, p / 64].
+ *   block_table    device int32 [batch, max_pages]
+ *   kv_cache       device, fmt-dependent (see above), [num_blocks, 64, ...],
+ *                  16-byte aligned; only the slots of the new tokens change
+ *   fmt            MLA_KV_BF16: the 1,152 bytes of each token are stored as
+ *                  given.  MLA_KV_FP8_656: per 128-wide latent group g,
+ *                  scale_g = amax_g / 448 and code = E4M3 (OCP, bias 7)
+ *                  round-to-nearest-even of x / scale_g, saturated to +-448,
+ *                  both divisions IEEE binary32; a group with amax_g = 0 gets
+ *                  scale 0 and codes 0; the RoPE values are copied as bf16.
+ *   workspace      device buffer whose first 4 bytes are a status word (the
+ *                  decode workspace serves), >= 4 bytes, 4-byte aligned
+ * One kernel (a warp per new token) enqueued on `stream`.  Device-detected
+ * errors, recorded in the status word, with the token not written:
+ *   p < 0 (cache_seqlens[b] < s_new)                 MLA_ERR_INVALID_ARG
+ *   p / 64 >= max_pages, or a block index outside
+ *   [0, num_blocks)                                  MLA_ERR_BAD_BLOCK_INDEX
+ * Two new tokens that map to the same slot race; the result is one of them.
+ */
+mla_status_t mla_kv_append(const void* kv_new, int batch, int s_new, const int32_t* cache_seqlens,
+                           const int32_t* block_table, int max_pages, void* kv_cache, mla_kv_format_t fmt,
+                           int64_t num_blocks, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device-detected status recorded in
  * `workspace` (MLA_OK if none) or MLA_ERR_CUDA if the stream reports an error. */
 mla_status_t mla_last_device_status(const void* workspace, void* stream);

@@ -7,7 +7,7 @@ or the device is not an sm_100 part, calls raise.
 
 Names follow the C ABI:
   mla_default_num_sm_parts, mla_metadata_size, mla_get_metadata,
-  mla_workspace_size, mla_decode_fwd, mla_last_device_status,
+  mla_workspace_size, mla_decode_fwd, mla_kv_append, mla_last_device_status,
   mla_clear_device_status, mla_status_string
 plus `decode(...)`, a convenience wrapper that allocates the outputs, the
 schedule and the workspace.
@@ -60,6 +60,8 @@ def load_library():
     lib.mla_decode_fwd.restype = c_int
     lib.mla_decode_fwd.argtypes = [vp, vp, c_int, c_i64, vp, c_int, vp, c_int, c_int, c_int, c_float, c_int,
                                    vp, vp, c_int, vp, vp, vp, c_size, vp]
+    lib.mla_kv_append.restype = c_int
+    lib.mla_kv_append.argtypes = [vp, c_int, c_int, vp, vp, c_int, vp, c_int, c_i64, vp, c_size, vp]
     lib.mla_last_device_status.restype = c_int
     lib.mla_last_device_status.argtypes = [vp, vp]
     lib.mla_clear_device_status.restype = c_int
@@ -144,6 +146,24 @@ def mla_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_tabl
                               out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
                               _stream(stream)), "mla_decode_fwd")
     return out, lse
+
+
+def mla_kv_append(kv_new: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_table: torch.Tensor,
+                  cache_seqlens: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """Enqueue the append of kv_new (bf16 [batch, s_new, 576]) into the paged cache on `stream`.
+
+    cache_seqlens are the lengths after the append; new token t of request b
+    lands at position cache_seqlens[b] - s_new + t (see include/mla.h).
+    """
+    lib = load_library()
+    B, s_new, d = kv_new.shape
+    assert d == 576 and kv_new.dtype == torch.bfloat16 and kv_new.is_contiguous()
+    assert kv_cache.is_contiguous() and block_table.is_contiguous() and block_table.dtype == torch.int32
+    assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
+    _check(lib.mla_kv_append(kv_new.data_ptr(), B, s_new, cache_seqlens.data_ptr(), block_table.data_ptr(),
+                             block_table.shape[1], kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
+                             workspace.data_ptr(), workspace.numel(), _stream(stream)), "mla_kv_append")
+    return kv_cache
 
 
 def mla_last_device_status(workspace: torch.Tensor, stream=None) -> int:

@@ -7,7 +7,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SOURCES = ["api.cu", "decode.cu", "metadata.cu", "combine.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "decode.cu", "metadata.cu", "combine.cu", "noalloc.cu", "append.cu"]
 OUT = os.path.join(HERE, "libmla_b200.so")
 
 
@@ -20,7 +20,7 @@ def nvcc_path() -> str:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(HERE, "csrc", s) for s in SOURCES]
-    deps = srcs + [os.path.join(HERE, "csrc", h) for h in ("common.cuh", "sm100.cuh")] + \
+    deps = srcs + [os.path.join(HERE, "csrc", h) for h in ("common.cuh", "sm100.cuh", "append.cuh")] + \
         [os.path.join(HERE, "..", "include", "mla.h")]
     if not force and os.path.exists(OUT) and all(os.path.getmtime(OUT) >= os.path.getmtime(d) for d in deps):
         return OUT

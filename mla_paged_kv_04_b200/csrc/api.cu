@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "../../include/mla.h"
+#include "append.cuh"
 #include "common.cuh"
 
 namespace mla {
@@ -198,6 +199,35 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
   c.num_parts = num_sm_parts;
   e = launch_combine(c, num_sm_parts, s);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_kv_append(const void* kv_new, int batch, int s_new, const int32_t* cache_seqlens,
+                           const int32_t* block_table, int max_pages, void* kv_cache, mla_kv_format_t fmt,
+                           int64_t num_blocks, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!kv_new || !cache_seqlens || !block_table || !kv_cache || !workspace) return MLA_ERR_INVALID_ARG;
+  if (!aligned(kv_new, 16) || !aligned(kv_cache, 16) || !aligned(block_table, 4) || !aligned(cache_seqlens, 4) ||
+      !aligned(workspace, 4))
+    return MLA_ERR_INVALID_ARG;
+  if (fmt != MLA_KV_BF16 && fmt != MLA_KV_FP8_656) return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || s_new < 1 || max_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || num_blocks > (static_cast<int64_t>(1) << 31) / kPage) return MLA_ERR_INVALID_ARG;
+  // one warp per token, eight per block: the grid stays below 2^31 blocks
+  const long long tokens = static_cast<long long>(batch) * s_new;
+  if (tokens > (static_cast<long long>(1) << 33)) return MLA_ERR_UNSUPPORTED;
+  if (workspace_bytes < sizeof(int)) return MLA_ERR_WORKSPACE;
+  if (!device_supported()) return MLA_ERR_UNSUPPORTED;
+  AppendParams p{};
+  p.kv_new = static_cast<const uint16_t*>(kv_new);
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.kv_cache = static_cast<uint8_t*>(kv_cache);
+  p.status = static_cast<int*>(workspace);
+  p.num_blocks = num_blocks;
+  p.tokens = tokens;
+  p.max_pages = max_pages;
+  p.s_new = s_new;
+  p.fp8 = fmt == MLA_KV_FP8_656 ? 1 : 0;
+  return launch_append(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status_t mla_last_device_status(const void* workspace, void* stream) {

@@ -82,6 +82,33 @@ def test_decode_argument_validation(lib):
     assert _call_decode(lib, ws_bytes=1024) == WORKSPACE
 
 
+def _call_append(lib, **over):
+    args = dict(new=16, batch=2, s_new=1, seqlens=16, bt=16, max_pages=4, kv=16, fmt=1, num_blocks=10, ws=16,
+                ws_bytes=256, stream=None)
+    args.update(over)
+    return lib.mla_kv_append(args["new"], args["batch"], args["s_new"], args["seqlens"], args["bt"],
+                             args["max_pages"], args["kv"], args["fmt"], args["num_blocks"], args["ws"],
+                             args["ws_bytes"], args["stream"])
+
+
+def test_append_argument_validation(lib):
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+    assert _call_append(lib, new=None) == INVALID
+    assert _call_append(lib, kv=None) == INVALID
+    assert _call_append(lib, ws=None) == INVALID
+    assert _call_append(lib, new=8) == INVALID           # misaligned rows
+    assert _call_append(lib, kv=4) == INVALID
+    assert _call_append(lib, seqlens=2) == INVALID
+    assert _call_append(lib, fmt=3) == INVALID
+    assert _call_append(lib, batch=0) == INVALID
+    assert _call_append(lib, s_new=0) == INVALID
+    assert _call_append(lib, max_pages=0) == INVALID
+    assert _call_append(lib, num_blocks=0) == INVALID
+    assert _call_append(lib, num_blocks=1 << 30) == INVALID
+    assert _call_append(lib, batch=1 << 30, s_new=1 << 10) == UNSUPPORTED
+    assert _call_append(lib, ws_bytes=2) == WORKSPACE
+
+
 def test_metadata_argument_validation(lib):
     INVALID, UNSUPPORTED = 1, 2
     f = lib.mla_get_metadata
