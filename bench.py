@@ -224,12 +224,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The maximum of x over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(units_per_rank: float, ms_per_step_max: float, world: int) -> float:
+    """Whole-job rate: the units all ranks processed per second of the slowest
+    rank's time (weak scaling: every rank runs its own replica)."""
+    return world * units_per_rank / (ms_per_step_max * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -402,8 +410,8 @@ def run_cuda(args, world, rank, local):
     peaks = load_peaks()
     n = world
     ms_per_step = total_ms / args.steps
-    value = n * work["bytes"] / (ms_per_step * 1e-3) / 1e9
-    tflops = n * work["flops"] / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_rate(work["bytes"], ms_per_step, n) / 1e9
+    tflops = aggregate_rate(work["flops"], ms_per_step, n) / 1e12
     dec_avg = statistics.mean(dec_ms)
     achieved = work["bytes"] / (dec_avg * 1e-3) / 1e9
     compute_bound = work["flops"] / work["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -563,7 +571,7 @@ def run_append(args, world, rank, local):
         gbs, sample, cores = oracle_append_rate(w)
         cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {
-        "metric": APPEND_METRIC, "value": n * work / (ms_per_step * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": n,
+        "metric": APPEND_METRIC, "value": aggregate_rate(work, ms_per_step, n) / 1e9, "unit": "GB/s", "n_gpus": n,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.fmt == "bf16" else "f32",
         "data": "synthetic",
