@@ -7,7 +7,7 @@ or the device is not an sm_100 part, calls raise.
 
 Names follow the C ABI:
   mla_default_num_sm_parts, mla_metadata_size, mla_get_metadata,
-  mla_workspace_size, mla_decode_fwd, mla_kv_append, mla_last_device_status,
+  mla_workspace_size, mla_decode_fwd, mla_decode_fwd_noalloc, mla_kv_append, mla_last_device_status,
   mla_clear_device_status, mla_status_string
 plus `decode(...)`, a convenience wrapper that allocates the outputs, the
 schedule and the workspace.
@@ -60,6 +60,9 @@ def load_library():
     lib.mla_decode_fwd.restype = c_int
     lib.mla_decode_fwd.argtypes = [vp, vp, c_int, c_i64, vp, c_int, vp, c_int, c_int, c_int, c_float, c_int,
                                    vp, vp, c_int, vp, vp, vp, c_size, vp]
+    lib.mla_decode_fwd_noalloc.restype = c_int
+    lib.mla_decode_fwd_noalloc.argtypes = [vp, vp, c_int, c_i64, vp, c_int, vp, c_int, c_int, c_int, c_float, c_int,
+                                           vp, vp, c_int, vp, vp, vp]
     lib.mla_kv_append.restype = c_int
     lib.mla_kv_append.argtypes = [vp, c_int, c_int, vp, vp, c_int, vp, c_int, c_i64, vp, c_size, vp]
     lib.mla_last_device_status.restype = c_int
@@ -145,6 +148,26 @@ def mla_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_tabl
                               1 if causal else 0, sched.data_ptr(), num_splits.data_ptr(), int(num_sm_parts),
                               out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
                               _stream(stream)), "mla_decode_fwd")
+    return out, lse
+
+
+def mla_decode_fwd_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_table: torch.Tensor,
+                           cache_seqlens: torch.Tensor, softmax_scale: float, causal: bool, sched: torch.Tensor,
+                           num_splits: torch.Tensor, num_sm_parts: int, out: torch.Tensor, lse: torch.Tensor,
+                           stream=None):
+    """mla_decode_fwd without a workspace: the split-KV scratch is the library's
+    static per-device array (see include/mla.h for its size limit and sharing)."""
+    lib = load_library()
+    B, s_q, h_q, d = q.shape
+    assert d == 576 and q.dtype == torch.bfloat16 and q.is_contiguous()
+    assert kv_cache.is_contiguous() and block_table.is_contiguous() and block_table.dtype == torch.int32
+    assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
+    assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
+    _check(lib.mla_decode_fwd_noalloc(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
+                                      block_table.data_ptr(), block_table.shape[1], cache_seqlens.data_ptr(), B, s_q,
+                                      h_q, float(softmax_scale), 1 if causal else 0, sched.data_ptr(),
+                                      num_splits.data_ptr(), int(num_sm_parts), out.data_ptr(), lse.data_ptr(),
+                                      _stream(stream)), "mla_decode_fwd_noalloc")
     return out, lse
 
 
