@@ -84,6 +84,19 @@ def _check(status: int, where: str):
         raise MLAError(status, where)
 
 
+def _check_cache(kv_cache: torch.Tensor, fmt: str):
+    """The cache tensor must be what `fmt` says, since the kernels address it
+    as [num_blocks, 64, token bytes] from its first dimension alone."""
+    if fmt not in FORMATS:
+        raise ValueError(f"unknown cache format {fmt!r}")
+    want = (torch.bfloat16, 576) if fmt == "bf16" else (torch.uint8, 656)
+    if kv_cache.dtype != want[0] or kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (64, want[1]):
+        raise ValueError(f"{fmt} cache must be {want[0]} [num_blocks, 64, {want[1]}], "
+                         f"got {kv_cache.dtype} {tuple(kv_cache.shape)}")
+    if not kv_cache.is_contiguous():
+        raise ValueError("the cache must be contiguous")
+
+
 def mla_status_string(status: int) -> str:
     return load_library().mla_status_string(status).decode()
 
@@ -139,7 +152,8 @@ def mla_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_tabl
     lib = load_library()
     B, s_q, h_q, d = q.shape
     assert d == 576 and q.dtype == torch.bfloat16 and q.is_contiguous()
-    assert kv_cache.is_contiguous() and block_table.is_contiguous() and block_table.dtype == torch.int32
+    _check_cache(kv_cache, fmt)
+    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
     assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
     assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
     num_blocks = kv_cache.shape[0]
@@ -160,7 +174,8 @@ def mla_decode_fwd_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, bl
     lib = load_library()
     B, s_q, h_q, d = q.shape
     assert d == 576 and q.dtype == torch.bfloat16 and q.is_contiguous()
-    assert kv_cache.is_contiguous() and block_table.is_contiguous() and block_table.dtype == torch.int32
+    _check_cache(kv_cache, fmt)
+    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
     assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
     assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
     _check(lib.mla_decode_fwd_noalloc(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
@@ -181,7 +196,8 @@ def mla_kv_append(kv_new: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_
     lib = load_library()
     B, s_new, d = kv_new.shape
     assert d == 576 and kv_new.dtype == torch.bfloat16 and kv_new.is_contiguous()
-    assert kv_cache.is_contiguous() and block_table.is_contiguous() and block_table.dtype == torch.int32
+    _check_cache(kv_cache, fmt)
+    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
     assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
     _check(lib.mla_kv_append(kv_new.data_ptr(), B, s_new, cache_seqlens.data_ptr(), block_table.data_ptr(),
                              block_table.shape[1], kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],

@@ -126,3 +126,18 @@ def test_product_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def test_binding_rejects_a_cache_that_does_not_match_its_format():
+    import torch
+    import mla_paged_kv_04_b200 as mla
+    mla._check_cache(torch.zeros((2, 64, 576), dtype=torch.bfloat16), "bf16")
+    mla._check_cache(torch.zeros((2, 64, 656), dtype=torch.uint8), "fp8_656")
+    for bad, fmt in [(torch.zeros((2, 64, 576), dtype=torch.uint8), "bf16"),
+                     (torch.zeros((2, 64, 656), dtype=torch.uint8), "bf16"),
+                     (torch.zeros((2, 64, 576), dtype=torch.bfloat16), "fp8_656"),
+                     (torch.zeros((2, 32, 656), dtype=torch.uint8), "fp8_656"),
+                     (torch.zeros((2, 576, 64), dtype=torch.bfloat16).transpose(1, 2), "bf16"),
+                     (torch.zeros((2, 64, 576), dtype=torch.bfloat16), "fp16")]:
+        with pytest.raises(ValueError):
+            mla._check_cache(bad, fmt)
