@@ -156,11 +156,12 @@ def mla_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_tabl
     assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
     assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
     assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
+    assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
     num_blocks = kv_cache.shape[0]
     _check(lib.mla_decode_fwd(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], num_blocks, block_table.data_ptr(),
                               block_table.shape[1], cache_seqlens.data_ptr(), B, s_q, h_q, float(softmax_scale),
                               1 if causal else 0, sched.data_ptr(), num_splits.data_ptr(), int(num_sm_parts),
-                              out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                              out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                               _stream(stream)), "mla_decode_fwd")
     return out, lse
 
@@ -178,6 +179,7 @@ def mla_decode_fwd_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, bl
     assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
     assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
     assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
+    assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
     _check(lib.mla_decode_fwd_noalloc(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
                                       block_table.data_ptr(), block_table.shape[1], cache_seqlens.data_ptr(), B, s_q,
                                       h_q, float(softmax_scale), 1 if causal else 0, sched.data_ptr(),
@@ -201,7 +203,7 @@ def mla_kv_append(kv_new: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_
     assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
     _check(lib.mla_kv_append(kv_new.data_ptr(), B, s_new, cache_seqlens.data_ptr(), block_table.data_ptr(),
                              block_table.shape[1], kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
-                             workspace.data_ptr(), workspace.numel(), _stream(stream)), "mla_kv_append")
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream)), "mla_kv_append")
     return kv_cache
 
 
