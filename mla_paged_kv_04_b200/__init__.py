@@ -161,8 +161,8 @@ def mla_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_tabl
     _check(lib.mla_decode_fwd(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], num_blocks, block_table.data_ptr(),
                               block_table.shape[1], cache_seqlens.data_ptr(), B, s_q, h_q, float(softmax_scale),
                               1 if causal else 0, sched.data_ptr(), num_splits.data_ptr(), int(num_sm_parts),
-                              out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                              _stream(stream)), "mla_decode_fwd")
+                              out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream(stream)), "mla_decode_fwd")
     return out, lse
 
 
@@ -203,7 +203,8 @@ def mla_kv_append(kv_new: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_
     assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
     _check(lib.mla_kv_append(kv_new.data_ptr(), B, s_new, cache_seqlens.data_ptr(), block_table.data_ptr(),
                              block_table.shape[1], kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
-                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream)), "mla_kv_append")
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream)),
+           "mla_kv_append")
     return kv_cache
 
 
