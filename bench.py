@@ -8,16 +8,29 @@ CUDA events on the launching stream.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
   python bench.py --op append [--workload NAME]   (the cache-append kernel, see run_append)
+  python bench.py --trace [--workload NAME] [--batch B]   (per-phase cycles, trace build)
 
-Prints ONE JSON line on rank 0.  Under torchrun each rank runs an independent
-replica of the workload (requests are independent, there is no data-path
-collective); the time is the max over ranks and `value` aggregates all ranks.
-`--impl reference` times the float64 CPU oracle on a bounded sample instead.
+Prints ONE JSON line on rank 0.  By default the line's top-level numbers are
+those of the FP8 656-byte-cache workload (b=128, h_q=128, L ~ U[16384, 32768],
+the compute-bound configuration) in TFLOP/s, and `per_config` holds the same
+record for the four other workloads.  For each workload:
+  value        algorithmic flops / (time of the K timed steps / K)
+  roofline     the decode call alone (decode + combine kernels), median of at
+               least 50 calls each after an L2 flush, against the measured
+               peak of the bound (tensor or HBM)
+  e2e          through the public API with inputs uploaded from pinned host
+               memory and results downloaded every step
+  cpu_baseline the float64 oracle on the host cores, bounded sample
+Under torchrun each rank runs an independent replica of the workloads
+(requests are independent, there is no data-path collective); the time is the
+max over ranks and `value` aggregates all ranks.  `--impl reference` times the
+float64 CPU oracle on a bounded sample instead.
 """
 
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -36,7 +49,6 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "MLA decode TFLOPS & effective HBM GB/s on 1 B200 (frac of roofline)"
-DEFAULT_WORKLOAD = "uniform_bf16"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -167,35 +179,50 @@ class ClockSampler:
 # the CPU oracle as a timed baseline (bounded sample)
 # ---------------------------------------------------------------------------
 
+def oracle_threads() -> int:
+    """Threads the oracle's numpy BLAS runs with (what `cores` reports)."""
+    try:
+        from threadpoolctl import threadpool_info
+        return max([d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def oracle_rate(w: W.Workload, budget_s: float = 12.0, seed: int = 0):
     """Time the float64 oracle on whole requests of the workload until `budget_s`.
 
-    Returns (GB/s of algorithmic bytes, sample description, cores used).
+    The sample is fixed: four single requests drawn with the workload's
+    recipe (seeds seed .. seed + 3), cycled in order; one untimed call first
+    (page faults of the first allocation).  Returns ({"tflops", "gbs"} of
+    algorithmic work per second of oracle time, sample description, BLAS
+    threads).
     """
     import oracle
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
-    except Exception:
-        cores = os.cpu_count()
-    # whole requests of the workload, generated once on the CPU with its recipe
-    # and cycled until the time budget is spent
     pool = []
     for b in range(4):
         one = W.Workload(w.name, 1, w.s_q, w.h_q, w.seqlen, fmt=w.fmt, causal=w.causal, seed=seed + b)
         a = W.oracle_arrays(W.make_case(one, poison=False))
-        pool.append((a, algorithmic_work(one, a["cache_seqlens"])["bytes"]))
-    n_done, t_total, bytes_done = 0, 0.0, 0
-    while t_total < budget_s and n_done < 4096:
-        a, nbytes = pool[n_done % len(pool)]
-        t0 = time.perf_counter()
+        work = algorithmic_work(one, a["cache_seqlens"])
+        pool.append((a, work["bytes"], work["flops"]))
+
+    def call(a):
         oracle.mla_decode(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
                           a["softmax_scale"], a["causal"])
+
+    call(pool[0][0])
+    n_done, t_total, bytes_done, flops_done = 0, 0.0, 0, 0
+    while t_total < budget_s and n_done < 4096:
+        a, nbytes, nflops = pool[n_done % len(pool)]
+        t0 = time.perf_counter()
+        call(a)
         t_total += time.perf_counter() - t0
         bytes_done += nbytes
+        flops_done += nflops
         n_done += 1
-    sample = f"{n_done} whole requests of {w.describe()} ({t_total:.1f} s of oracle time)"
-    return bytes_done / t_total / 1e9, sample, cores, t_total / max(n_done, 1)
+    sample = (f"{n_done} whole requests of {w.describe()} cycled from 4 drawn with seeds {seed}..{seed + 3} "
+              f"({t_total:.1f} s of oracle time)")
+    return ({"tflops": flops_done / t_total / 1e12, "gbs": bytes_done / t_total / 1e9}, sample,
+            oracle_threads())
 
 
 # ---------------------------------------------------------------------------
@@ -245,40 +272,50 @@ def aggregate_rate(units_per_rank: float, ms_per_step_max: float, world: int) ->
 # ---------------------------------------------------------------------------
 
 def run_reference(args, world, rank):
+    """The reference arm: the float64 oracle on the host cores, on the same
+    workload, metric and unit as the CUDA arm's line, each step a bounded
+    sample of whole requests.  Rank 0 only."""
     if rank != 0:
         return
-    w = W.WORKLOADS[args.workload]
-    per_step = []
-    rate_bytes = 0
+    w = W.WORKLOADS[args.workload or HEADLINE]
+    per_step, gbs = [], []
     budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    sample = ""
+    cores = oracle_threads()
     for i in range(args.warmup + args.steps):
-        gbs, sample, cores, _ = oracle_rate(w, budget_s=budget, seed=1000 * i)
+        rate, sample, cores = oracle_rate(w, budget_s=budget, seed=0)
         if i >= args.warmup:
-            per_step.append(gbs)
+            per_step.append(rate["tflops"])
+            gbs.append(rate["gbs"])
     value = statistics.mean(per_step)
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.describe(), "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
                        "seqlen": list(w.seqlen), "kv_format": w.fmt},
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "gbs": statistics.mean(gbs),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": f"each step: {sample}"},
-            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_cuda(args, world, rank, local):
+HEADLINE = "fp8_656"          # the compute-bound configuration (FP8 656-byte cache)
+PER_CONFIG = ["tiny", "uniform_bf16", "varlen_spec_bf16", "long_ctx_bf16"]
+MIN_REPS = 50                 # decode calls timed for the roofline, at least
+REPS_SECONDS = 1.0            # ... and about this long, so that clocks are sampled under load
+
+
+def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: float, sampler_gpu: int):
+    """Everything bench.py reports for one workload on this rank.
+
+    Returns (record, total_ms_of_the_K_steps) where record holds the rank's
+    numbers; the caller takes the max over ranks of the step time.
+    """
     import mla_paged_kv_04_b200 as mla
-    from mla_paged_kv_04_b200 import build
-    if rank == 0:
-        build.build()
-    barrier(world)
-    mla.load_library()
-    w = W.WORKLOADS[args.workload]
-    dev = torch.device("cuda", local if world > 1 else 0)
     case = W.make_case(w, seed=w.seed + rank, device=dev, poison=False)
     q, kv, bt, L = case["q"], case["kv_cache"], case["block_table"], case["cache_seqlens"]
-    B, s_q, h_q = w.batch, w.s_q, w.h_q
+    B, s_q, h_q = case["batch"], w.s_q, w.h_q
     parts = args.parts or mla.mla_default_num_sm_parts(dev)
     sched = torch.empty(mla.mla_metadata_size(B, parts) // 4, dtype=torch.int32, device=dev)
     ns = torch.empty(B + 1, dtype=torch.int32, device=dev)
@@ -290,59 +327,72 @@ def run_cuda(args, world, rank, local):
     work = algorithmic_work(w, seqlens_np)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def meta():
         mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
+
+    def decode():
         mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
                            stream=stream)
 
-    for _ in range(args.warmup):
+    for _ in range(max(args.warmup, 3)):
         flush.zero_()
-        step()
+        meta()
+        decode()
     torch.cuda.synchronize(dev)
     status = mla.mla_last_device_status(ws)
     if status != 0:
-        raise SystemExit(f"device status {mla.STATUS.get(status, status)} during warm-up")
+        raise SystemExit(f"{w.name}: device status {mla.STATUS.get(status, status)} during warm-up")
+
+    # Time one decode call alone (for reps sizing).
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.zero_()
+    meta()
+    e0.record(stream)
+    decode()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    one_ms = max(e0.elapsed_time(e1), 1e-3)
+    reps = max(MIN_REPS, min(4000, int(REPS_SECONDS * 1e3 / (one_ms + 0.05))))
 
     # The timed steps: one event pair per step around the whole hot path
-    # (schedule + decode + combine).  No event sits between the kernels, so
-    # the decode kernel's programmatic early launch overlaps the schedule
-    # kernel's tail as it would in a serving loop.
+    # (schedule + decode + combine), L2 flushed before each.  No event sits
+    # between the kernels, so the decode kernel's programmatic early launch
+    # overlaps the schedule kernel's tail as it would in a serving loop.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    dec_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+    meta_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(MIN_REPS)]
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index or 0) as clk:
+    with ClockSampler(sampler_gpu) as clk:
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
-            step()
+            meta()
+            decode()
             ev[i][1].record(stream)
+        # The decode call alone (decode + combine kernels), for the roofline:
+        # the median of `reps` calls, each after an L2 flush and the schedule.
+        for i in range(reps):
+            flush.zero_()
+            meta()
+            dec_ev[i][0].record(stream)
+            decode()
+            dec_ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
     step_ms = [e[0].elapsed_time(e[1]) for e in ev]
     total_ms = max_over_ranks(sum(step_ms), world)
+    dec_ms = [e[0].elapsed_time(e[1]) for e in dec_ev]
+    for i in range(MIN_REPS):  # the schedule kernel alone
+        flush.zero_()
+        meta_ev[i][0].record(stream)
+        meta()
+        meta_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    meta_ms = [e[0].elapsed_time(e[1]) for e in meta_ev]
     status = mla.mla_last_device_status(ws)
     if status != 0:
-        raise SystemExit(f"device status {mla.STATUS.get(status, status)} in the timed region")
-
-    # The decode call alone (decode + combine kernels, for the roofline), and
-    # the schedule kernel alone, each timed over the same number of steps.
-    dec_ms, meta_ms = [], []
-    for i in range(args.steps):
-        flush.zero_()
-        mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
-        e1, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e1.record(stream)
-        mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
-                           stream=stream)
-        e2.record(stream)
-        flush.zero_()
-        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        m0.record(stream)
-        mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
-        m1.record(stream)
-        torch.cuda.synchronize(dev)
-        dec_ms.append(e1.elapsed_time(e2))
-        meta_ms.append(m0.elapsed_time(m1))
+        raise SystemExit(f"{w.name}: device status {mla.STATUS.get(status, status)} in the timed region")
 
     # End to end through the public API: every step uploads its inputs (q,
     # block table, sequence lengths) from pinned host memory, flushes L2, runs
@@ -390,69 +440,142 @@ def run_cuda(args, world, rank, local):
             lse_h[k].copy_(lse_d[k], non_blocking=True)
             dn_done[k].record(s_dn)
 
-    for i in range(args.warmup):
+    for i in range(max(args.warmup, 3)):
         e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier(world)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(s_up)
-    for i in range(args.warmup, args.warmup + args.steps):
+    w0 = max(args.warmup, 3)
+    for i in range(w0, w0 + args.steps):
         e2e_step(i)
     e_end.record(s_dn)
     torch.cuda.synchronize(dev)
     e2e_total = max_over_ranks(e_start.elapsed_time(e_end), world)
     status = mla.mla_last_device_status(ws)
     if status != 0:
-        raise SystemExit(f"device status {mla.STATUS.get(status, status)} in the end-to-end steps")
+        raise SystemExit(f"{w.name}: device status {mla.STATUS.get(status, status)} in the end-to-end steps")
 
-    if rank != 0:
-        return
-    peaks = load_peaks()
     n = world
     ms_per_step = total_ms / args.steps
-    value = aggregate_rate(work["bytes"], ms_per_step, n) / 1e9
-    tflops = aggregate_rate(work["flops"], ms_per_step, n) / 1e12
-    dec_avg = statistics.mean(dec_ms)
-    achieved = work["bytes"] / (dec_avg * 1e-3) / 1e9
-    compute_bound = work["flops"] / work["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if compute_bound:
-        ach_tf = work["flops"] / (dec_avg * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": ach_tf / peaks["bf16_tflops"], "traffic": None}
+    dec_med = statistics.median(dec_ms)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if work["flops"] / work["bytes"] > ridge:
+        ach = work["flops"] / (dec_med * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"]}
     else:
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
-    roof.update({"kernel": "decode (+ split-KV combine) via mla_decode_fwd", "peak_source": peaks["source"],
-                 "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"],
-                 "avg_ms": dec_avg})
-    roof["traffic"] = recorded_traffic(w.name)
-
+        ach = work["bytes"] / (dec_med * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"]}
+    roof.update({"traffic": recorded_traffic(w.name) if args.batch is None else None,
+                 "kernel": "decode (+ split-KV combine) via mla_decode_fwd",
+                 "peak_source": f"{peaks['source']} (burst)", "algorithmic_bytes": work["bytes"],
+                 "algorithmic_flops": work["flops"], "median_ms": dec_med, "reps": reps,
+                 "min_ms": min(dec_ms), "tflops": work["flops"] / (dec_med * 1e-3) / 1e12,
+                 "gbs": work["bytes"] / (dec_med * 1e-3) / 1e9})
+    e2e_ms = e2e_total / args.steps
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
-        gbs, sample, cores, _ = oracle_rate(w, budget_s=args.cpu_budget)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample}
-
-    clocks = clk.summary()
-    line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.describe(), "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
-                   "seqlen": list(w.seqlen), "kv_format": w.fmt, "causal": w.causal, "num_sm_parts": parts,
-                   "l2": "flushed before every timed step (256 MiB write)",
-                   "parallelism": f"replicas x{n} (independent request batches)"},
-        "tflops": tflops,
-        "metadata_ms": statistics.mean(meta_ms),
-        "roofline": roof,
-        "cpu_baseline": cpu,
-        "e2e": {"value": n * work["bytes"] / (e2e_total / args.steps * 1e-3) / 1e9, "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_total / args.steps,
+    if world == 1 and cpu_budget > 0:
+        rate, sample, cores = oracle_rate(w, budget_s=cpu_budget)
+        cpu = {"value": rate["tflops"], "unit": "TFLOP/s", "gbs": rate["gbs"], "cores": cores, "kind": "oracle",
+               "sample": sample}
+    rec = {
+        "workload": w.describe(), "value": aggregate_rate(work["flops"], ms_per_step, n) / 1e12,
+        "unit": "TFLOP/s", "gbs": aggregate_rate(work["bytes"], ms_per_step, n) / 1e9,
+        "ms_per_step": ms_per_step, "metadata_ms": statistics.median(meta_ms),
+        "config": {"workload": w.describe(), "batch": B, "s_q": w.s_q, "h_q": w.h_q, "seqlen": list(w.seqlen),
+                   "kv_format": w.fmt, "causal": w.causal, "num_sm_parts": parts},
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": n * work["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "gbs": n * work["bytes"] / (e2e_ms * 1e-3) / 1e9,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "uploads, kernels (with the L2 flush) and downloads of consecutive steps "
                               "overlap on three streams, two buffers deep"},
         "gpu_launches": 3 * args.steps,
-        "clocks": clocks,
+        "clocks": clk.summary(),
+    }
+    del case, q, kv, bt, L, ws, out, lse, flush, q_d, bt_d, L_d, out_d, lse_d
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_cuda(args, world, rank, local):
+    import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    mla.load_library()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    peaks = load_peaks()
+    head = W.WORKLOADS[args.workload or HEADLINE]
+    if args.batch is not None:
+        head = dataclasses.replace(head, batch=args.batch)
+    others = [] if (args.workload or args.batch is not None) else [W.WORKLOADS[n] for n in PER_CONFIG]
+    cpu_head = 0.0 if args.no_cpu_baseline else args.cpu_budget
+    cpu_other = 0.0 if args.no_cpu_baseline else min(3.0, args.cpu_budget)
+    rec = measure_workload(head, args, world, rank, dev, peaks, cpu_head, dev.index or 0)
+    per = {}
+    for w in others:
+        per[w.name] = measure_workload(w, args, world, rank, dev, peaks, cpu_other, dev.index or 0)
+    if rank != 0:
+        return
+    n = world
+    line = {
+        "metric": METRIC, "value": rec["value"], "unit": rec["unit"], "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(rec["config"], **{
+            "mma": "bf16 operands (FP8 cache dequantised in shared memory), fp32 accumulation",
+            "l2": "flushed before every timed step and every roofline rep (256 MiB write)",
+            "parallelism": f"replicas x{n} (independent request batches)"}),
+        "gbs": rec["gbs"],
+        "metadata_ms": rec["metadata_ms"],
+        "roofline": rec["roofline"],
+        "cpu_baseline": rec["cpu_baseline"],
+        "e2e": rec["e2e"],
+        "gpu_launches": rec["gpu_launches"],
+        "clocks": rec["clocks"],
+        "per_config": per,
     }
     print(json.dumps(line), flush=True)
+
+
+def run_trace(args):
+    """One decode call of the workload through the trace build; prints the
+    median length of each pipeline phase in SM cycles (and saves the raw
+    timestamps with --trace-out)."""
+    import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import build, trace
+    build.build(trace=True)
+    mla.load_library(trace=True)
+    w = W.WORKLOADS[args.workload or HEADLINE]
+    if args.batch is not None:
+        w = dataclasses.replace(w, batch=args.batch)
+    dev = torch.device("cuda", 0)
+    case = W.make_case(w, device=dev, poison=False)
+    q, kv, bt, L = case["q"], case["kv_cache"], case["block_table"], case["cache_seqlens"]
+    B = case["batch"]
+    parts = args.parts or mla.mla_default_num_sm_parts(dev)
+    sched, ns = mla.mla_get_metadata(L, w.s_q, w.h_q, parts)
+    ws = mla.alloc_workspace(B, w.s_q, w.h_q, parts, dev)
+    out = torch.empty((B, w.s_q, w.h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, w.s_q, w.h_q), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def run():
+        flush.zero_()
+        mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws)
+
+    for _ in range(3):
+        run()
+    ts = trace.record(run)
+    status = mla.mla_last_device_status(ws)
+    if args.trace_out:
+        np.save(args.trace_out, ts)
+    print(f"# {w.describe()}, {parts} CTA pairs, device status {mla.STATUS.get(status, status)}")
+    print(trace.format_summary(trace.summarize(ts)))
 
 
 # ---------------------------------------------------------------------------
@@ -497,7 +620,7 @@ def run_append(args, world, rank, local):
         build.build()
     barrier(world)
     mla.load_library()
-    w = W.WORKLOADS[args.workload]
+    w = W.WORKLOADS[args.workload or HEADLINE]
     dev = torch.device("cuda", local if world > 1 else 0)
     case = W.make_case(w, seed=w.seed + rank, device=dev, poison=False)
     kv, bt, L = case["kv_cache"], case["block_table"], case["cache_seqlens"]
@@ -596,17 +719,25 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=list(W.WORKLOADS),
+                    help=f"measure only this workload (default: {HEADLINE} as the headline, "
+                         f"the others under per_config)")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling runs)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--parts", type=int, default=0, help="CTA pairs (default: SMs / 2)")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="decode", choices=["decode", "append"])
+    ap.add_argument("--trace", action="store_true", help="per-tile phase timings from the trace build")
+    ap.add_argument("--trace-out", default=None, help="with --trace: save the raw timestamps (.npy)")
     args = ap.parse_args()
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, world, rank)
+        return
+    if args.trace:
+        run_trace(args)
         return
     world, rank, local = dist_setup(args.gpus)
     try:

@@ -129,6 +129,11 @@ size_t mla_workspace_size(int batch, int s_q, int h_q, int num_sm_parts);
  * only issue L2 prefetch hints for q and block_table, which read no value.)
  * Tail slots of a request's last page
  * and blocks it does not reference may hold any bits (NaN/Inf included).
+ * Device-detected errors (status word, see mla_last_device_status):
+ *   a block_table entry outside [0, num_blocks)     MLA_ERR_BAD_BLOCK_INDEX
+ *   sched made for another batch or num_sm_parts    MLA_ERR_INVALID_ARG
+ *     (nothing is computed or written then)
+ *   a wait that ran past its limit                  MLA_ERR_TIMEOUT
  */
 mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt,
                             int64_t num_blocks, const int32_t* block_table, int max_pages,
@@ -181,6 +186,47 @@ mla_status_t mla_last_device_status(const void* workspace, void* stream);
 mla_status_t mla_clear_device_status(void* workspace, void* stream);
 
 /*
+ * Diagnostics.  The pages have no counterpart of these calls.
+ *
+ * mla_set_wait_timeout_ns: every wait inside the decode kernel (for a page,
+ * for the tensor cores, for the peer CTA) gives up after this many
+ * nanoseconds; the kernel then records MLA_ERR_TIMEOUT in the status word,
+ * drains its copies and tensor-core work, frees its tensor memory and exits,
+ * leaving out/lse undefined.  The default is 2 s, far above any legitimate
+ * wait; a smaller value lets a test or a watchdog see that path.  Applies to
+ * decode calls enqueued after it returns, process-wide; 0 restores the
+ * default.  Returns the previous value.
+ */
+uint64_t mla_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * mla_debug_set_trace_buffer: only a library built with MLA_TRACE defined
+ * (build.py builds it as libmla_b200_trace.so) records per-tile timestamps of
+ * the decode kernel: for the first 4 CTAs and their first 128 tiles, the SM
+ * clock at fixed points of each warp role (layout in csrc/common.cuh), into
+ * a caller-owned device buffer of mla_debug_trace_bytes() bytes, 8-byte
+ * aligned.  NULL stops recording.  The product library returns
+ * MLA_ERR_UNSUPPORTED and records nothing.
+ */
+size_t mla_debug_trace_bytes(void);
+mla_status_t mla_debug_set_trace_buffer(void* buffer, size_t bytes);
+
+/*
+ * mla_debug_hold_at_tile: from the next decode call on (process-wide), the
+ * thread of every CTA that issues the P*V tensor-core work waits, before the
+ * tile it counts as number `tile` (from 0, over the CTA's whole run), until
+ * the device int at `flag` becomes non-zero.  That wait is bounded like every
+ * other one (mla_set_wait_timeout_ns).  With a flag that nothing sets, the
+ * wait runs out while the pipeline is full, and the call ends through the
+ * abort path: MLA_ERR_TIMEOUT in the status word, copies and tensor-core work
+ * drained, tensor memory freed, the context still usable.  This is how the
+ * tests exercise failure detection without faulting a GPU.  flag NULL or
+ * tile < 0 turns the hold off (the default).  `flag` must be 4-byte aligned
+ * and stay valid while decode calls that may hold on it run.
+ */
+mla_status_t mla_debug_hold_at_tile(const int* flag, int tile);
+
+/*
  * Allocation-free decode.  The pages have no counterpart of this call: it is a
  * deployment aid of this library for callers that cannot allocate device
  * memory or pass a workspace, e.g. code running during CUDA graph capture,
@@ -191,17 +237,18 @@ mla_status_t mla_clear_device_status(void* workspace, void* stream);
  * split-KV scratch (status word + partial results) lives in a static array
  * of MLA_NOALLOC_SCRATCH_BYTES inside the library, reserved on every GPU that
  * loads the library until the process exits.  The call allocates nothing.
- *   - Returns MLA_ERR_WORKSPACE, enqueuing nothing, when the shape needs more
- *     scratch than that, i.e. mla_workspace_size(batch, s_q, h_q,
- *     num_sm_parts) > MLA_NOALLOC_SCRATCH_BYTES (64 MiB: for 128 query rows
- *     per request, batch + num_sm_parts <= 255).
+ *   - Argument errors return the same codes as mla_decode_fwd, enqueuing
+ *     nothing.  MLA_ERR_WORKSPACE, also with nothing enqueued, when the shape
+ *     needs more scratch than the array holds, i.e. mla_workspace_size(batch,
+ *     s_q, h_q, num_sm_parts) > MLA_NOALLOC_SCRATCH_BYTES (64 MiB: for 128
+ *     query rows per request, batch + num_sm_parts <= 255).
  *   - The first call on a device (with that device current) looks up the
  *     array's device address; make that first call before any stream capture.
  *   - All calls share the one array and it keeps the previous call's contents;
  *     each call resets the status word on `stream` first.  Calls that can
  *     overlap on the GPU (other streams or host threads) race on the array.
- * Device-detected errors are recorded in the shared array and are not
- * reported by this call.
+ * Device-detected errors go to the status word inside the shared array;
+ * mla_noalloc_last_device_status reads it (for the current device).
  */
 #define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
 mla_status_t mla_decode_fwd_noalloc(const void* q, const void* kv_cache, mla_kv_format_t fmt,
@@ -210,6 +257,11 @@ mla_status_t mla_decode_fwd_noalloc(const void* q, const void* kv_cache, mla_kv_
                                     float softmax_scale, int causal, const int32_t* sched,
                                     const int32_t* num_splits, int num_sm_parts, void* out,
                                     float* lse, void* stream);
+
+/* Synchronises `stream`, then returns the device-detected status of the last
+ * mla_decode_fwd_noalloc call on the current device (MLA_OK if none was
+ * recorded).  The next call on the device clears it. */
+mla_status_t mla_noalloc_last_device_status(void* stream);
 
 #ifdef __cplusplus
 }

@@ -7,10 +7,13 @@ or the device is not an sm_100 part, calls raise.
 
 Names follow the C ABI:
   mla_default_num_sm_parts, mla_metadata_size, mla_get_metadata,
-  mla_workspace_size, mla_decode_fwd, mla_decode_fwd_noalloc, mla_kv_append, mla_last_device_status,
-  mla_clear_device_status, mla_status_string
+  mla_workspace_size, mla_decode_fwd, mla_decode_fwd_noalloc,
+  mla_noalloc_last_device_status, mla_kv_append, mla_last_device_status,
+  mla_clear_device_status, mla_status_string, mla_set_wait_timeout_ns,
+  mla_debug_trace_bytes, mla_debug_set_trace_buffer, mla_debug_hold_at_tile
 plus `decode(...)`, a convenience wrapper that allocates the outputs, the
-schedule and the workspace.
+schedule and the workspace.  Every tensor argument is checked (device, dtype,
+shape, size) before its pointer reaches the C ABI.
 """
 
 from __future__ import annotations
@@ -22,6 +25,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+TRACE_LIB_PATH = os.path.join(_HERE, "libmla_b200_trace.so")
 
 MLA_KV_BF16 = 0
 MLA_KV_FP8_656 = 1
@@ -30,6 +34,7 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
           4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_BAD_BLOCK_INDEX"}
 
 _lib = None
+_trace_lib = None
 
 
 class MLAError(RuntimeError):
@@ -38,14 +43,19 @@ class MLAError(RuntimeError):
         super().__init__(f"{where}: {STATUS.get(status, status)}")
 
 
-def load_library():
-    """Load libmla_b200.so (built in-tree by `build.build()`); raise if absent."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with mla_paged_kv_04_b200.build.build()")
-    lib = ctypes.CDLL(LIB_PATH)
+def load_library(trace: bool = False):
+    """Load libmla_b200.so (built in-tree by `build.build()`); raise if absent.
+
+    trace=True loads the timestamp-recording build (libmla_b200_trace.so,
+    `build.build(trace=True)`) instead; see trace.py.
+    """
+    global _lib, _trace_lib
+    if (_trace_lib if trace else _lib) is not None:
+        return _trace_lib if trace else _lib
+    path = TRACE_LIB_PATH if trace else LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with mla_paged_kv_04_b200.build.build(trace={trace})")
+    lib = ctypes.CDLL(path)
     c_int, c_size, vp, c_float, c_i64 = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float, ctypes.c_int64
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_status_string.argtypes = [c_int]
@@ -69,8 +79,29 @@ def load_library():
     lib.mla_last_device_status.argtypes = [vp, vp]
     lib.mla_clear_device_status.restype = c_int
     lib.mla_clear_device_status.argtypes = [vp, vp]
-    _lib = lib
+    lib.mla_noalloc_last_device_status.restype = c_int
+    lib.mla_noalloc_last_device_status.argtypes = [vp]
+    lib.mla_set_wait_timeout_ns.restype = ctypes.c_uint64
+    lib.mla_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.mla_debug_trace_bytes.restype = c_size
+    lib.mla_debug_trace_bytes.argtypes = []
+    lib.mla_debug_set_trace_buffer.restype = c_int
+    lib.mla_debug_set_trace_buffer.argtypes = [vp, c_size]
+    lib.mla_debug_hold_at_tile.restype = c_int
+    lib.mla_debug_hold_at_tile.argtypes = [vp, c_int]
+    if trace:
+        _trace_lib = lib
+    else:
+        _lib = lib
     return lib
+
+
+def _active_lib():
+    """The library the calls go through: the product one, unless only the
+    trace build has been loaded (trace.py does that)."""
+    if _lib is None and _trace_lib is not None:
+        return _trace_lib
+    return load_library()
 
 
 def _stream(stream=None) -> int:
@@ -82,6 +113,51 @@ def _stream(stream=None) -> int:
 def _check(status: int, where: str):
     if status != 0:
         raise MLAError(status, where)
+
+
+def _on_device(device: torch.device, **tensors):
+    """Every tensor must live on `device` (a CUDA device) and be contiguous:
+    the C ABI receives bare pointers and cannot tell."""
+    if device.type != "cuda":
+        raise ValueError(f"tensors must be CUDA tensors, got {device}")
+    for name, t in tensors.items():
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
+def _check_decode_tensors(q, kv_cache, fmt, block_table, cache_seqlens, sched, num_splits, num_sm_parts, out,
+                          lse, workspace=None):
+    """Shapes, dtypes, devices and sizes of a decode call's tensors."""
+    if q.dim() != 4 or q.shape[3] != 576 or q.dtype != torch.bfloat16:
+        raise ValueError(f"q must be bf16 [batch, s_q, h_q, 576], got {q.dtype} {tuple(q.shape)}")
+    B, s_q, h_q, _ = q.shape
+    tensors = dict(q=q, kv_cache=kv_cache, block_table=block_table, cache_seqlens=cache_seqlens, sched=sched,
+                   num_splits=num_splits, out=out, lse=lse)
+    if workspace is not None:
+        tensors["workspace"] = workspace
+    _on_device(q.device, **tensors)
+    _check_cache(kv_cache, fmt)
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be int32 [batch={B}, max_pages], got {block_table.dtype} "
+                         f"{tuple(block_table.shape)}")
+    if cache_seqlens.dtype != torch.int32 or cache_seqlens.numel() != B:
+        raise ValueError(f"cache_seqlens must be int32 [{B}]")
+    if out.shape != (B, s_q, h_q, 512) or out.dtype != torch.bfloat16:
+        raise ValueError(f"out must be bf16 {(B, s_q, h_q, 512)}, got {out.dtype} {tuple(out.shape)}")
+    if lse.shape != (B, s_q, h_q) or lse.dtype != torch.float32:
+        raise ValueError(f"lse must be fp32 {(B, s_q, h_q)}, got {lse.dtype} {tuple(lse.shape)}")
+    if sched.dtype != torch.int32 or _nbytes(sched) < mla_metadata_size(B, int(num_sm_parts)):
+        raise ValueError(f"sched must be int32 of >= mla_metadata_size({B}, {num_sm_parts}) bytes")
+    if num_splits.dtype != torch.int32 or num_splits.numel() < B + 1:
+        raise ValueError(f"num_splits must be int32 [>= {B + 1}]")
 
 
 def _check_cache(kv_cache: torch.Tensor, fmt: str):
@@ -98,30 +174,31 @@ def _check_cache(kv_cache: torch.Tensor, fmt: str):
 
 
 def mla_status_string(status: int) -> str:
-    return load_library().mla_status_string(status).decode()
+    return _active_lib().mla_status_string(status).decode()
 
 
 def mla_default_num_sm_parts(device=None) -> int:
     dev = torch.cuda.current_device() if device is None else torch.device(device).index or 0
-    n = load_library().mla_default_num_sm_parts(dev)
+    n = _active_lib().mla_default_num_sm_parts(dev)
     if n <= 0:
         raise MLAError(4, "mla_default_num_sm_parts")
     return n
 
 
 def mla_metadata_size(batch: int, num_sm_parts: int) -> int:
-    return load_library().mla_metadata_size(batch, num_sm_parts)
+    return _active_lib().mla_metadata_size(batch, num_sm_parts)
 
 
 def mla_workspace_size(batch: int, s_q: int, h_q: int, num_sm_parts: int) -> int:
-    return load_library().mla_workspace_size(batch, s_q, h_q, num_sm_parts)
+    return _active_lib().mla_workspace_size(batch, s_q, h_q, num_sm_parts)
 
 
 def mla_get_metadata(cache_seqlens: torch.Tensor, s_q: int, h_q: int, num_sm_parts: int | None = None,
                      sched: torch.Tensor | None = None, num_splits: torch.Tensor | None = None, stream=None):
     """Split-KV schedule for `cache_seqlens` (device int32 [batch]) -> (sched, num_splits)."""
-    lib = load_library()
-    assert cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous()
+    lib = _active_lib()
+    if not cache_seqlens.is_cuda or cache_seqlens.dtype != torch.int32:
+        raise ValueError("cache_seqlens must be a CUDA int32 tensor")
     batch = cache_seqlens.numel()
     parts = mla_default_num_sm_parts(cache_seqlens.device) if num_sm_parts is None else int(num_sm_parts)
     nbytes = lib.mla_metadata_size(batch, parts)
@@ -129,7 +206,10 @@ def mla_get_metadata(cache_seqlens: torch.Tensor, s_q: int, h_q: int, num_sm_par
         sched = torch.empty(max(nbytes // 4, 1), dtype=torch.int32, device=cache_seqlens.device)
     if num_splits is None:
         num_splits = torch.empty(batch + 1, dtype=torch.int32, device=cache_seqlens.device)
-    if sched.numel() * 4 < nbytes:
+    _on_device(cache_seqlens.device, cache_seqlens=cache_seqlens, sched=sched, num_splits=num_splits)
+    if sched.dtype != torch.int32 or num_splits.dtype != torch.int32 or num_splits.numel() < batch + 1:
+        raise ValueError(f"sched and num_splits must be int32, num_splits of >= {batch + 1} entries")
+    if _nbytes(sched) < nbytes:
         raise MLAError(3, "mla_get_metadata")
     _check(lib.mla_get_metadata(cache_seqlens.data_ptr(), batch, s_q, h_q, parts, sched.data_ptr(),
                                 num_splits.data_ptr(), _stream(stream)), "mla_get_metadata")
@@ -149,20 +229,16 @@ def mla_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_tabl
                    num_splits: torch.Tensor, num_sm_parts: int, out: torch.Tensor, lse: torch.Tensor,
                    workspace: torch.Tensor, stream=None):
     """Enqueue the decode (and, where needed, the split-KV combine) on `stream`."""
-    lib = load_library()
-    B, s_q, h_q, d = q.shape
-    assert d == 576 and q.dtype == torch.bfloat16 and q.is_contiguous()
-    _check_cache(kv_cache, fmt)
-    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
-    assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
-    assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
-    assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
+    lib = _active_lib()
+    _check_decode_tensors(q, kv_cache, fmt, block_table, cache_seqlens, sched, num_splits, num_sm_parts, out, lse,
+                          workspace)
+    B, s_q, h_q, _ = q.shape
     num_blocks = kv_cache.shape[0]
     _check(lib.mla_decode_fwd(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], num_blocks, block_table.data_ptr(),
                               block_table.shape[1], cache_seqlens.data_ptr(), B, s_q, h_q, float(softmax_scale),
                               1 if causal else 0, sched.data_ptr(), num_splits.data_ptr(), int(num_sm_parts),
                               out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
-                              workspace.numel() * workspace.element_size(), _stream(stream)), "mla_decode_fwd")
+                              _nbytes(workspace), _stream(stream)), "mla_decode_fwd")
     return out, lse
 
 
@@ -172,20 +248,54 @@ def mla_decode_fwd_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, bl
                            stream=None):
     """mla_decode_fwd without a workspace: the split-KV scratch is the library's
     static per-device array (see include/mla.h for its size limit and sharing)."""
-    lib = load_library()
-    B, s_q, h_q, d = q.shape
-    assert d == 576 and q.dtype == torch.bfloat16 and q.is_contiguous()
-    _check_cache(kv_cache, fmt)
-    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
-    assert out.shape == (B, s_q, h_q, 512) and out.dtype == torch.bfloat16 and out.is_contiguous()
-    assert lse.shape == (B, s_q, h_q) and lse.dtype == torch.float32 and lse.is_contiguous()
-    assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
+    lib = _active_lib()
+    _check_decode_tensors(q, kv_cache, fmt, block_table, cache_seqlens, sched, num_splits, num_sm_parts, out, lse)
+    B, s_q, h_q, _ = q.shape
     _check(lib.mla_decode_fwd_noalloc(q.data_ptr(), kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
                                       block_table.data_ptr(), block_table.shape[1], cache_seqlens.data_ptr(), B, s_q,
                                       h_q, float(softmax_scale), 1 if causal else 0, sched.data_ptr(),
                                       num_splits.data_ptr(), int(num_sm_parts), out.data_ptr(), lse.data_ptr(),
                                       _stream(stream)), "mla_decode_fwd_noalloc")
     return out, lse
+
+
+def mla_noalloc_last_device_status(stream=None) -> int:
+    """Synchronise the stream and return the device status of the last
+    mla_decode_fwd_noalloc call on the current device (0 = MLA_OK)."""
+    return _active_lib().mla_noalloc_last_device_status(_stream(stream))
+
+
+def mla_set_wait_timeout_ns(ns: int) -> int:
+    """Limit of every wait inside later decode kernels (0 = the 2 s default);
+    returns the previous limit."""
+    return int(_active_lib().mla_set_wait_timeout_ns(int(ns)))
+
+
+def mla_debug_trace_bytes() -> int:
+    return int(_active_lib().mla_debug_trace_bytes())
+
+
+def mla_debug_set_trace_buffer(buffer: torch.Tensor | None) -> int:
+    """Point the trace build's timestamp recording at `buffer` (None stops it).
+    Returns the status (MLA_ERR_UNSUPPORTED from the product library)."""
+    lib = _active_lib()
+    if buffer is None:
+        return lib.mla_debug_set_trace_buffer(None, 0)
+    _on_device(buffer.device, buffer=buffer)
+    return lib.mla_debug_set_trace_buffer(buffer.data_ptr(), _nbytes(buffer))
+
+
+def mla_debug_hold_at_tile(flag: torch.Tensor | None, tile: int = -1):
+    """Make later decode calls wait at tile `tile` until the device int32
+    `flag` is non-zero (bounded by the wait timeout); None turns it off."""
+    lib = _active_lib()
+    if flag is None:
+        _check(lib.mla_debug_hold_at_tile(None, -1), "mla_debug_hold_at_tile")
+        return
+    _on_device(flag.device, flag=flag)
+    if flag.dtype != torch.int32 or flag.numel() < 1:
+        raise ValueError("flag must be a device int32 tensor")
+    _check(lib.mla_debug_hold_at_tile(flag.data_ptr(), int(tile)), "mla_debug_hold_at_tile")
 
 
 def mla_kv_append(kv_new: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_table: torch.Tensor,
@@ -195,26 +305,33 @@ def mla_kv_append(kv_new: torch.Tensor, kv_cache: torch.Tensor, fmt: str, block_
     cache_seqlens are the lengths after the append; new token t of request b
     lands at position cache_seqlens[b] - s_new + t (see include/mla.h).
     """
-    lib = load_library()
-    B, s_new, d = kv_new.shape
-    assert d == 576 and kv_new.dtype == torch.bfloat16 and kv_new.is_contiguous()
+    lib = _active_lib()
+    if kv_new.dim() != 3 or kv_new.shape[2] != 576 or kv_new.dtype != torch.bfloat16:
+        raise ValueError(f"kv_new must be bf16 [batch, s_new, 576], got {kv_new.dtype} {tuple(kv_new.shape)}")
+    B, s_new, _ = kv_new.shape
+    _on_device(kv_new.device, kv_new=kv_new, kv_cache=kv_cache, block_table=block_table,
+               cache_seqlens=cache_seqlens, workspace=workspace)
     _check_cache(kv_cache, fmt)
-    assert block_table.is_contiguous() and block_table.dtype == torch.int32 and block_table.shape[0] == B
-    assert cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous() and cache_seqlens.numel() == B
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be int32 [batch={B}, max_pages]")
+    if cache_seqlens.dtype != torch.int32 or cache_seqlens.numel() != B:
+        raise ValueError(f"cache_seqlens must be int32 [{B}]")
     _check(lib.mla_kv_append(kv_new.data_ptr(), B, s_new, cache_seqlens.data_ptr(), block_table.data_ptr(),
                              block_table.shape[1], kv_cache.data_ptr(), FORMATS[fmt], kv_cache.shape[0],
-                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream)),
+                             workspace.data_ptr(), _nbytes(workspace), _stream(stream)),
            "mla_kv_append")
     return kv_cache
 
 
 def mla_last_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise the stream and return the device status code (0 = MLA_OK)."""
-    return load_library().mla_last_device_status(workspace.data_ptr(), _stream(stream))
+    _on_device(workspace.device, workspace=workspace)
+    return _active_lib().mla_last_device_status(workspace.data_ptr(), _stream(stream))
 
 
 def mla_clear_device_status(workspace: torch.Tensor, stream=None):
-    _check(load_library().mla_clear_device_status(workspace.data_ptr(), _stream(stream)), "mla_clear_device_status")
+    _on_device(workspace.device, workspace=workspace)
+    _check(_active_lib().mla_clear_device_status(workspace.data_ptr(), _stream(stream)), "mla_clear_device_status")
 
 
 def decode(q, kv_cache, block_table, cache_seqlens, softmax_scale, causal=False, fmt="bf16", num_sm_parts=None,

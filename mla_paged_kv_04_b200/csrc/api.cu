@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -12,6 +13,7 @@
 #include "../../include/mla.h"
 #include "append.cuh"
 #include "common.cuh"
+#include "entry.cuh"
 
 namespace mla {
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int parts, int32_t* sched, int32_t* num_splits,
@@ -29,6 +31,15 @@ using namespace mla;
 namespace {
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+// Limit of every bounded wait in the decode kernel (mla_set_wait_timeout_ns).
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+// Timestamp buffer of a trace build (mla_debug_set_trace_buffer), else null.
+std::atomic<unsigned long long*> g_trace{nullptr};
+// mla_debug_hold_at_tile: the flag (null = off) and the tile.
+std::mutex g_hold_mutex;
+const int* g_hold_flag = nullptr;
+int g_hold_tile = -1;
 
 bool aligned(const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
@@ -77,6 +88,25 @@ mla_status_t check_shape(int batch, int s_q, int h_q) {
 
 }  // namespace
 
+namespace mla {
+
+// Synchronises the stream, then maps the status word at `word` (device) to
+// an mla_status_t.
+mla_status_t read_device_status(const void* word, void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
+  switch (status) {
+    case 0: return MLA_OK;
+    case kStatusBadSchedule: return MLA_ERR_INVALID_ARG;
+    case kStatusTimeout: return MLA_ERR_TIMEOUT;
+    case kStatusBadBlock: return MLA_ERR_BAD_BLOCK_INDEX;
+    default: return MLA_ERR_CUDA;
+  }
+}
+
+}  // namespace mla
+
 extern "C" {
 
 const char* mla_status_string(mla_status_t s) {
@@ -120,27 +150,38 @@ size_t mla_workspace_size(int batch, int s_q, int h_q, int num_sm_parts) {
   return ws_bytes(batch, num_sm_parts, s_q * h_q);
 }
 
-mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt, int64_t num_blocks,
-                            const int32_t* block_table, int max_pages, const int32_t* cache_seqlens, int batch,
-                            int s_q, int h_q, float softmax_scale, int causal, const int32_t* sched,
-                            const int32_t* num_splits, int num_sm_parts, void* out, float* lse, void* workspace,
-                            size_t workspace_bytes, void* stream) {
-  if (!q || !kv_cache || !block_table || !cache_seqlens || !sched || !num_splits || !out || !lse || !workspace)
+}  // extern "C"
+
+namespace mla {
+
+// Everything about a decode call the host can check, except the workspace
+// and the device.
+mla_status_t check_decode_args(const void* q, const void* kv_cache, mla_kv_format_t fmt, int64_t num_blocks,
+                               const int32_t* block_table, int max_pages, const int32_t* cache_seqlens, int batch,
+                               int s_q, int h_q, float softmax_scale, const int32_t* sched,
+                               const int32_t* num_splits, int num_sm_parts, const void* out, const float* lse) {
+  if (!q || !kv_cache || !block_table || !cache_seqlens || !sched || !num_splits || !out || !lse)
     return MLA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(kv_cache, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
-      !aligned(block_table, 4) || !aligned(cache_seqlens, 4) || !aligned(lse, 4) || !aligned(sched, 16) ||
-      !aligned(num_splits, 4))
+  if (!aligned(q, 16) || !aligned(kv_cache, 16) || !aligned(out, 16) || !aligned(block_table, 4) ||
+      !aligned(cache_seqlens, 4) || !aligned(lse, 4) || !aligned(sched, 16) || !aligned(num_splits, 4))
     return MLA_ERR_INVALID_ARG;
   if (fmt != MLA_KV_BF16 && fmt != MLA_KV_FP8_656) return MLA_ERR_INVALID_ARG;
   if (num_blocks < 1 || num_blocks > (static_cast<int64_t>(1) << 31) / kPage) return MLA_ERR_INVALID_ARG;
   if (max_pages < 1 || num_sm_parts < 1 || num_sm_parts > 65535) return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
-  mla_status_t st = check_shape(batch, s_q, h_q);
-  if (st != MLA_OK) return st;
-  const int M = s_q * h_q;
-  if (workspace_bytes < ws_bytes(batch, num_sm_parts, M)) return MLA_ERR_WORKSPACE;
-  if (!device_supported()) return MLA_ERR_UNSUPPORTED;
+  return check_shape(batch, s_q, h_q);
+}
 
+bool current_device_supported() { return device_supported(); }
+
+// Enqueues the decode and combine kernels of a call whose arguments passed
+// check_decode_args and whose workspace holds ws_bytes(batch, parts, M).
+mla_status_t launch_decode_call(const void* q, const void* kv_cache, mla_kv_format_t fmt, int64_t num_blocks,
+                                const int32_t* block_table, int max_pages, const int32_t* cache_seqlens, int batch,
+                                int s_q, int h_q, float softmax_scale, int causal, const int32_t* sched,
+                                const int32_t* num_splits, int num_sm_parts, void* out, float* lse, void* workspace,
+                                void* stream) {
+  const int M = s_q * h_q;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   DecodeParams p{};
@@ -162,7 +203,13 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
   p.causal = causal ? 1 : 0;
   p.num_parts = num_sm_parts;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
-  p.timeout_ns = kDefaultTimeoutNs;
+  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  p.trace = g_trace.load(std::memory_order_relaxed);
+  {
+    std::lock_guard<std::mutex> lock(g_hold_mutex);
+    p.hold_flag = g_hold_flag;
+    p.hold_tile = g_hold_tile;
+  }
 
   const uint64_t rows = static_cast<uint64_t>(num_blocks) * kPage;
   CUtensorMap tm_a, tm_b, tm_c;
@@ -201,6 +248,25 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+}  // namespace mla
+
+extern "C" {
+
+mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t fmt, int64_t num_blocks,
+                            const int32_t* block_table, int max_pages, const int32_t* cache_seqlens, int batch,
+                            int s_q, int h_q, float softmax_scale, int causal, const int32_t* sched,
+                            const int32_t* num_splits, int num_sm_parts, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = check_decode_args(q, kv_cache, fmt, num_blocks, block_table, max_pages, cache_seqlens, batch,
+                                      s_q, h_q, softmax_scale, sched, num_splits, num_sm_parts, out, lse);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes < ws_bytes(batch, num_sm_parts, s_q * h_q)) return MLA_ERR_WORKSPACE;
+  if (!device_supported()) return MLA_ERR_UNSUPPORTED;
+  return launch_decode_call(q, kv_cache, fmt, num_blocks, block_table, max_pages, cache_seqlens, batch, s_q, h_q,
+                            softmax_scale, causal, sched, num_splits, num_sm_parts, out, lse, workspace, stream);
+}
+
 mla_status_t mla_kv_append(const void* kv_new, int batch, int s_new, const int32_t* cache_seqlens,
                            const int32_t* block_table, int max_pages, void* kv_cache, mla_kv_format_t fmt,
                            int64_t num_blocks, void* workspace, size_t workspace_bytes, void* stream) {
@@ -232,17 +298,33 @@ mla_status_t mla_kv_append(const void* kv_new, int batch, int s_new, const int32
 
 mla_status_t mla_last_device_status(const void* workspace, void* stream) {
   if (!workspace) return MLA_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return MLA_ERR_CUDA;
-  int status = 0;
-  if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MLA_ERR_CUDA;
-  switch (status) {
-    case 0: return MLA_OK;
-    case kStatusBadSchedule: return MLA_ERR_INVALID_ARG;
-    case kStatusTimeout: return MLA_ERR_TIMEOUT;
-    case kStatusBadBlock: return MLA_ERR_BAD_BLOCK_INDEX;
-    default: return MLA_ERR_CUDA;
-  }
+  return read_device_status(workspace, stream);
+}
+
+uint64_t mla_set_wait_timeout_ns(uint64_t ns) {
+  return g_timeout_ns.exchange(ns == 0 ? kDefaultTimeoutNs : ns);
+}
+
+size_t mla_debug_trace_bytes(void) { return kTraceBytes; }
+
+mla_status_t mla_debug_hold_at_tile(const int* flag, int tile) {
+  if (flag != nullptr && !aligned(flag, 4)) return MLA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_hold_mutex);
+  g_hold_flag = (tile < 0) ? nullptr : flag;
+  g_hold_tile = (flag == nullptr) ? -1 : tile;
+  return MLA_OK;
+}
+
+mla_status_t mla_debug_set_trace_buffer(void* buffer, size_t bytes) {
+#ifdef MLA_TRACE
+  if (buffer != nullptr && (bytes < kTraceBytes || !aligned(buffer, 8))) return MLA_ERR_INVALID_ARG;
+  g_trace.store(static_cast<unsigned long long*>(buffer));
+  return MLA_OK;
+#else
+  (void)buffer;
+  (void)bytes;
+  return MLA_ERR_UNSUPPORTED;
+#endif
 }
 
 mla_status_t mla_clear_device_status(void* workspace, void* stream) {

@@ -22,7 +22,9 @@ constexpr int kCombineUnroll = 4;  // splits whose partial rows are in flight at
 // kCombineUnroll splits are loaded together so that their latencies overlap.
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineParams p) {
   pdl_wait();  // the decode kernel has completed
-  if (p.sched[0] != p.num_parts) return;  // reported by the decode kernel
+  // a schedule made for another CTA-pair count or batch: reported by the
+  // decode kernel, nothing to merge
+  if (p.sched[0] != p.num_parts || p.sched[3] != p.batch) return;
   const int num_split_req = p.sched[5];
   if (static_cast<int>(blockIdx.x) >= num_split_req) return;
   const int parts = p.sched[0];

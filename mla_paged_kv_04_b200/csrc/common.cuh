@@ -81,7 +81,34 @@ struct DecodeParams {
   int num_parts;                // CTA pairs launched (must equal sched[0])
   float scale_log2;             // softmax_scale * log2(e)
   unsigned long long timeout_ns;
+  unsigned long long* trace;    // per-tile timestamps (trace build only), else null
+  const int* hold_flag;         // diagnostics (mla_debug_hold_at_tile): device flag, or null
+  int hold_tile;                // the PV issuer's tile at which it waits for *hold_flag != 0
 };
+
+// Per-tile timestamps of the decode kernel, recorded only by a library built
+// with MLA_TRACE: trace[cta][role][tile][slot] holds the SM clock (clock64)
+// when a role passed a fixed point of its loop, for the first kTraceCtas CTAs
+// and their first kTraceTiles tiles.  Role kTraceCta, tile 0, also holds the
+// global timer (ns) at kernel entry in slot 15, so that CTAs can be aligned.
+constexpr int kTraceCtas = 4;
+constexpr int kTraceRoles = 7;
+constexpr int kTraceTiles = 128;
+constexpr int kTraceSlots = 16;
+enum : int {
+  kTraceProducer = 0,  // 0 wait for a free stage, 1 copies issued
+  kTraceQk = 1,        // 0 wait for the page, 1 page ready, 2 S free, 3 issued
+  kTracePv = 2,        // 0 wait for P, 1 P ready, 2 issued
+  kTraceSoftmax = 3,   // 0 wait for S, 1 S ready, 2 S loaded, 3 row max, 4 buffer
+                       // credit, 5 sent, 6 first half in, 7 P formed, 8 reference
+                       // chain, 9 P buffer free, 10 O rescaled, 11 P stored
+  kTraceDequant = 4,   // 0 wait for raw bytes, 1 raw ready, 2 stage free, 3 done
+  kTraceItem = 5,      // tile = item: 0 start, 1 Q stored, 2 epilogue start, 3 done
+  kTraceCta = 6,       // tile 0: 0 entry, 1 set up, 2 schedule readable, 3 roles
+                       // done, 4 exit, 15 global timer at entry
+};
+constexpr size_t kTraceBytes =
+    sizeof(unsigned long long) * kTraceCtas * kTraceRoles * kTraceTiles * kTraceSlots;
 
 struct CombineParams {
   const int32_t* sched;         // schedule buffer (split-request list)

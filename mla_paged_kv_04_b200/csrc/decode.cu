@@ -50,6 +50,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -101,7 +103,8 @@ struct Cfg {
   static constexpr int kQRopeOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
   // [wg][row] fp32: each warpgroup's latest lazy reference; [row] the
   // combined reference of the last consumed tile; [wg][row] the row-sum parts
-  // at the item's final scale.  Then barriers, abort flag, tmem base.
+  // at the item's final scale.  Then barriers, the abort flag, the tensor-
+  // memory base and the slot where the peer CTA reports its abort flag.
   static constexpr int kRefSlotOffset = kQRopeOffset + kRows * 64;
   static constexpr int kCombSlotOffset = kRefSlotOffset + 2 * kRows * 4;
   static constexpr int kEpiOffset = kCombSlotOffset + kRows * 4;
@@ -120,6 +123,19 @@ constexpr uint32_t kColQ = 384;  // 128 columns: Q's 256 latent dims as packed b
 
 __device__ const int g_never_abort = 0;
 
+// Per-tile timestamps (layout in common.cuh).  Only a library compiled with
+// MLA_TRACE records them; the product build emits no code for TRACE.
+#ifdef MLA_TRACE
+__device__ __forceinline__ void trace_point(const DecodeParams& p, int role, uint32_t tile, int slot) {
+  if (p.trace != nullptr && blockIdx.x < static_cast<unsigned>(kTraceCtas) && tile < static_cast<uint32_t>(kTraceTiles))
+    p.trace[((static_cast<size_t>(blockIdx.x) * kTraceRoles + role) * kTraceTiles + tile) * kTraceSlots + slot] =
+        clock64();
+}
+#define TRACE(role, tile, slot) trace_point(p, (role), static_cast<uint32_t>(tile), (slot))
+#else
+#define TRACE(role, tile, slot) ((void)0)
+#endif
+
 // Warp-uniform bounded wait.  Fast path: every lane tries the phase once (a
 // completed phase, the common case, costs one warp-wide try).  Otherwise lane 0
 // polls with the time limit, then every lane performs its own (immediately
@@ -137,6 +153,22 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const v
       if (kCluster ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity)) break;
   }
   return ok != 0;
+}
+
+// Diagnostics (mla_debug_hold_at_tile): wait, bounded like every other wait,
+// until the host-visible flag becomes non-zero.  A test gives a flag that
+// nothing sets, so the wait runs out with the pipeline full and the abort
+// path (drain copies and MMAs, free tensor memory, report MLA_ERR_TIMEOUT)
+// runs for real.
+__device__ __forceinline__ bool hold_until_flag(const DecodeParams& p, const volatile int* abort_flag) {
+  const volatile int* flag = p.hold_flag;
+  const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+  while (*flag == 0) {
+    if (*abort_flag || globaltimer_ns() - t0 > p.timeout_ns) return false;
+    __nanosleep(256);
+  }
+  return true;
 }
 
 __device__ __forceinline__ void raise_abort(const DecodeParams& p, volatile int* abort_flag) {
@@ -170,6 +202,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   using C = Cfg<kFp8>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
+  TRACE(kTraceCta, 0, 0);
+#ifdef MLA_TRACE
+  if (threadIdx.x == 0 && p.trace != nullptr && blockIdx.x < static_cast<unsigned>(kTraceCtas))
+    p.trace[(static_cast<size_t>(blockIdx.x) * kTraceRoles + kTraceCta) * kTraceTiles * kTraceSlots + 15] =
+        globaltimer_ns();
+#endif
   // The combine kernel may start launching now; it waits for this grid.
   pdl_launch_dependents();
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -231,6 +269,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   cluster_sync();  // the peer's barriers are initialised before any st.async reaches them
+  if (threadIdx.x == 0) TRACE(kTraceCta, 0, 1);
 
   // While the schedule kernel finishes: start q and the block table towards
   // L2, spread over every thread of the grid, so that the first Q and
@@ -251,12 +290,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   // written by the previous kernel in the stream (mla_get_metadata), and the
   // workspace and outputs may still be read by the previous combine pass.
   pdl_wait();
+  if (threadIdx.x == 0) TRACE(kTraceCta, 0, 2);
   const int num_parts = p.sched[0];
   const int32_t* items = p.sched + sched_items_offset(num_parts);
   int it_begin = 0, it_end = 0;
-  if (num_parts != p.num_parts) {
-    // schedule made for another CTA-pair count: its item slots may not fit
-    // the workspace, so do nothing and report it
+  if (num_parts != p.num_parts || p.sched[3] != p.batch) {
+    // schedule made for another CTA-pair count or another batch: its request
+    // ids and item slots may lie outside this call's tensors and workspace,
+    // so do nothing and report it
     if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
   } else {
     it_begin = p.sched[kSchedHeader + part];
@@ -297,6 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         }
         for (int pg = p0; pg < p1; ++pg, ++g) {
           const uint32_t st = g % nst;
+          TRACE(kTraceProducer, g, 0);
           if (g >= static_cast<uint32_t>(nst) &&
               !mbar_wait(BAR(empty0 + st), ((g / nst) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
             raise_abort(p, abort_flag);
@@ -326,6 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
               tma_load_2d(dst + c * kChunkBytes, &tm_a, fb, static_cast<int>(rank) * 256 + c * 64, y);
             tma_load_2d(dst + 4 * kChunkBytes, &tm_b, fb, 512 + static_cast<int>(rank) * 32, y);
           }
+          TRACE(kTraceProducer, g, 1);
         }
       }
       // Never leave a copy landing in shared memory after the CTA exits.
@@ -350,8 +393,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         ++nitem;
         for (int j = 0; j < n; ++j, ++g) {
           const uint32_t st = g % kStages;
+          TRACE(kTraceQk, g, 0);
           if (!mbar_wait(BAR(C::kFull + st), (g / kStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          TRACE(kTraceQk, g, 1);
           if (g > 0 && !mbar_wait(BAR(C::kSFree), (g - 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          TRACE(kTraceQk, g, 2);
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>((st * kStageBytes) >> 4);
 #pragma unroll
@@ -361,6 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) mma_ss(tmem + kColS, d_qrope + 2 * ks, d_rope + so + 2 * ks, idesc_qk, 1u);
           tc_commit(BAR(C::kSFull + (g & 1u)));
+          TRACE(kTraceQk, g, 3);
         }
       }
       if (!ok) raise_abort(p, abort_flag);
@@ -379,7 +426,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const int n = items[4 * it + 2] - items[4 * it + 1];
         for (int j = 0; j < n; ++j, ++g) {
           const uint32_t pb = g & 1u;
+          TRACE(kTracePv, g, 0);
+          if (p.hold_flag != nullptr && static_cast<int>(g) == p.hold_tile && !hold_until_flag(p, abort_flag)) {
+            ok = false;
+            break;
+          }
           if (!mbar_wait(BAR(C::kPFull + pb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          TRACE(kTracePv, g, 1);
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>(((g % kStages) * kStageBytes) >> 4);
 #pragma unroll
@@ -388,6 +441,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
                    (j == 0 && ks == 0) ? 0u : 1u);
           tc_commit(BAR(C::kPvDone + pb));
           tc_commit(BAR(C::kEmpty + g % kStages));
+          TRACE(kTracePv, g, 2);
         }
       }
       if (!ok) raise_abort(p, abort_flag);
@@ -436,6 +490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         }
         continue;
       }
+      if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 0);
       // Q -> tensor memory: this CTA's 256 latent dims as 128 packed bf16
       // pairs (warpgroup w writes columns [64 w, 64 w + 64)); the 32 RoPE dims
       // go to shared memory (SW64 K-major rows of 64 bytes), warpgroup 1.
@@ -470,6 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kQReady));
+        if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 1);
       }
       const int vis = p.causal ? min(L, L - p.s_q + qi + 1) : L;
       // every row sees at least this many keys: tiles below it need no mask
@@ -486,13 +542,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         // ---------------------------------------------------------------- produce
         // read the partial logits of tile gg, fix the row's lazy reference,
         // exponentiate, send the fp16 factors (+ reference) to the peer CTA
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 0);
         if (!warp_wait(BAR(C::kSFull + (gg & 1u)), (gg >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 1);
         tc_fence_after();
         uint32_t s[64];
         tmem_ld64(trow + kColS, s);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kSFree));
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 2);
         const int tok0 = pg * kPage;
         const bool full_tile = tok0 + kPage <= vis_all;
         float e[64];
@@ -522,6 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         // the reference: this warpgroup's last one, raised to the other
         // warpgroup's latest (read without waiting; any value works, and the
         // two converge after a tile or two)
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 3);
         const float prev = fmaxf(ref_own, ref_slot[(wg ^ 1) * kRows + r]);
         const float ref = (tmax > prev + kRescaleThreshold) ? tmax : prev;
         ref_own = ref;
@@ -538,6 +598,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           ok = false;
           break;
         }
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 4);
         {
           // Exponentiate and send in two halves of 32 tokens: the first half
           // crosses to the peer while the second is computed.
@@ -567,6 +628,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           }
           st_async_b32(rx + kXERegionBytes + r * 4, __float_as_uint(ref), xbar_peer + 8u * (2 * xb + 1));
         }
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 5);
         // ---------------------------------------------------------------- consume
         // combine with the peer's factors into P, rescale O when the combined
         // reference moved, hand P to the PV MMA
@@ -582,6 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             ok = false;
             break;
           }
+          if (wt == 0 && h == 0) TRACE(kTraceSoftmax, gg, 6);
 #pragma unroll
           for (int c = 4 * h; c < 4 * h + 4; ++c) {
             const uint4 w = *reinterpret_cast<const uint4*>(xs + (c * kRows + r) * 16);
@@ -595,8 +658,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           }
         }
         if (!ok) break;
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 7);
         const float m_new = ref + *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
         if (gg > 0 && !warp_wait(BAR(C::kCChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 8);
         const float m_prev = j > 0 ? comb_slot[r] : -CUDART_INF_F;
         comb_slot[r] = m_new;
         mbar_arrive(BAR(C::kCChain));
@@ -613,6 +678,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           if (!warp_wait(BAR(C::kPvDone + pb), ((gg - 2) >> 1) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
         }
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 9);
         const bool moved = m_new != m_prev;
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
           // O must be stable: PV(gg - 1) done
@@ -633,6 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             tmem_st16(trow + col + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
           }
         }
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 10);
         if (m_new != m_l) {
           l = (m_l == -CUDART_INF_F) ? 0.f : l * ex2_approx(m_l - m_new);
           m_l = m_new;
@@ -659,10 +726,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::kPFull + pb));
+        if (wt == 0) TRACE(kTraceSoftmax, gg, 11);
       }
       if (!ok) break;
       // epilogue: both warpgroups' row sums at the combined reference of the
       // item's last tile, then this warpgroup's 128 columns of O
+      if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 2);
       const uint32_t glast = g + static_cast<uint32_t>(n) - 1u;
       g += static_cast<uint32_t>(n);
       float m_fin = m_l;  // this warpgroup consumed the last tile
@@ -713,6 +782,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (slot < 0) p.lse[orow] = lse_val;
         else p.lse_part[static_cast<size_t>(slot) * p.M + r] = lse_val;
       }
+      if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 3);
     }
     if (!ok) raise_abort(p, abort_flag);
     __syncwarp();
@@ -732,9 +802,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       const int last_page = (L - 1) / kPage;
       for (int pg = p0; pg < p1; ++pg, ++g) {
         const uint32_t rs = g % kRawStages, st = g % kStages;
+        if (dt == 0) TRACE(kTraceDequant, g, 0);
         if (!warp_wait(BAR(C::kRawFull + rs), (g / kRawStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (dt == 0) TRACE(kTraceDequant, g, 1);
         if (g >= static_cast<uint32_t>(kStages) &&
             !warp_wait(BAR(C::kEmpty + st), ((g / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (dt == 0) TRACE(kTraceDequant, g, 2);
         const int valid = (pg == last_page) ? L - pg * kPage : kPage;
         const uint8_t* rlat = sbase + C::kRawOffset + rs * kRawBytes;
         const uint8_t* rscale = rlat + kRawLatBytes;
@@ -772,6 +845,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           mbar_arrive(BAR(C::kFull + st));
           mbar_arrive(BAR(C::kRawEmpty + rs));
         }
+        if (dt == 0) TRACE(kTraceDequant, g, 3);
       }
     }
     if (!ok) raise_abort(p, abort_flag);
@@ -781,7 +855,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // the peer no longer writes into this CTA's exchange buffers
+  if (threadIdx.x == 0) TRACE(kTraceCta, 0, 3);
+  // Teardown.  In the normal path the peer has waited for every message this
+  // CTA sent it, so no transfer is in flight and one cluster barrier suffices.
+  // After an abort the peer may have stopped consuming, and distributed-
+  // shared-memory stores or remote arrives issued here may still be on their
+  // way to it.  Each CTA therefore tells the other whether it gave up; if
+  // either did, both let such transfers land (they take about a microsecond;
+  // the wait is 50 us) before a second cluster barrier, after which either
+  // CTA may exit and release its shared memory.
+  volatile int* peer_abort = reinterpret_cast<volatile int*>(sbase + C::kBarOffset + C::kNumBars * 8 + 8);
+  if (threadIdx.x == 0)
+    st_cluster_u32(mapa_shared(base + C::kBarOffset + C::kNumBars * 8 + 8, peer), static_cast<uint32_t>(*abort_flag));
+  cluster_sync();
+  if (*abort_flag != 0 || *peer_abort != 0) {
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+      for (int i = 0; i < 1000 && globaltimer_ns() - t0 < 50000ull; ++i) __nanosleep(1000);
+    }
+    __syncthreads();
+    cluster_sync();
+  }
+  if (threadIdx.x == 0) TRACE(kTraceCta, 0, 4);
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -793,12 +889,19 @@ template <bool kFp8>
 static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_c,
                                  const DecodeParams& p, int num_parts, cudaStream_t stream) {
   using C = dk::Cfg<kFp8>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+  // The shared-memory opt-in is an attribute of the function on each device:
+  // set it once per device (a bit per device below 64; devices above that set
+  // it on every launch).  Racing host threads may both set it, which is
+  // harmless.
+  static std::atomic<unsigned long long> attr_done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit == 0 || (attr_done.load(std::memory_order_acquire) & bit) == 0) {
+    e = cudaFuncSetAttribute(decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
   // Programmatic dependent launch: the CTAs start (barriers, tensor memory)
   // while the metadata kernel finishes, and wait in the kernel before

@@ -23,6 +23,7 @@
 
 #include "../../include/mla.h"
 #include "common.cuh"
+#include "entry.cuh"
 
 namespace {
 
@@ -58,17 +59,27 @@ mla_status_t mla_decode_fwd_noalloc(const void* q, const void* kv_cache, mla_kv_
                                     int batch, int s_q, int h_q, float softmax_scale, int causal,
                                     const int32_t* sched, const int32_t* num_splits, int num_sm_parts, void* out,
                                     float* lse, void* stream) {
-  const size_t need = mla_workspace_size(batch, s_q, h_q, num_sm_parts);
-  if (need == 0) return MLA_ERR_UNSUPPORTED;
-  if (need > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE;
+  // Every host-side check comes before anything is enqueued.
+  mla_status_t st = mla::check_decode_args(q, kv_cache, fmt, num_blocks, block_table, max_pages, cache_seqlens,
+                                           batch, s_q, h_q, softmax_scale, sched, num_splits, num_sm_parts, out, lse);
+  if (st != MLA_OK) return st;
+  if (mla::ws_bytes(batch, num_sm_parts, s_q * h_q) > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE;
+  if (!mla::current_device_supported()) return MLA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
-  mla_status_t st = scratch_for_current_device(&scratch);
+  st = scratch_for_current_device(&scratch);
   if (st != MLA_OK) return st;
   if (cudaMemsetAsync(scratch, 0, sizeof(int), static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MLA_ERR_CUDA;
-  return mla_decode_fwd(q, kv_cache, fmt, num_blocks, block_table, max_pages, cache_seqlens, batch, s_q, h_q,
-                        softmax_scale, causal, sched, num_splits, num_sm_parts, out, lse, scratch,
-                        kNoAllocScratchBytes, stream);
+  return mla::launch_decode_call(q, kv_cache, fmt, num_blocks, block_table, max_pages, cache_seqlens, batch, s_q,
+                                 h_q, softmax_scale, causal, sched, num_splits, num_sm_parts, out, lse, scratch,
+                                 stream);
+}
+
+mla_status_t mla_noalloc_last_device_status(void* stream) {
+  void* scratch = nullptr;
+  mla_status_t st = scratch_for_current_device(&scratch);
+  if (st != MLA_OK) return st;
+  return mla::read_device_status(scratch, stream);
 }
 
 }  // extern "C"

@@ -156,6 +156,11 @@ __device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t v, u
                ::"r"(remote_addr), "r"(v), "r"(remote_bar)
                : "memory");
 }
+// Plain 32-bit store into the shared memory of a CTA of the cluster (address
+// from mapa); ordered before a later barrier.cluster.arrive.release.
+__device__ __forceinline__ void st_cluster_u32(uint32_t remote_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote_addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }

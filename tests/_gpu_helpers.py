@@ -66,6 +66,27 @@ def oracle_for(case, requests=None, dequant_bf16=False):
     return res
 
 
+def oracle_chunked(case, dequant_bf16=False, chunk=16):
+    """Oracle outputs of every request of a (possibly full-size) case, computed
+    a few requests at a time on compact copies of their pages, so that host
+    memory stays bounded.  Returns out [B, s_q, h_q, 512], lse [B, s_q, h_q]."""
+    B = case["batch"]
+    out = np.zeros((B, case["s_q"], case["h_q"], 512))
+    lse = np.full((B, case["s_q"], case["h_q"]), -np.inf)
+    for b0 in range(0, B, chunk):
+        reqs = list(range(b0, min(B, b0 + chunk)))
+        a = W.oracle_arrays_for(case, reqs)
+        if dequant_bf16 and a["fmt"] == "fp8_656":
+            kv = fp8_cache_as_bf16(torch.from_numpy(a["kv_cache"]))
+            a["kv_cache"] = kv.view(torch.int16).numpy().view(np.uint16)
+            a["fmt"] = "bf16"
+        res = oracle.mla_decode_rows(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
+                                     a["softmax_scale"], a["causal"], reqs)
+        for b in reqs:
+            out[b], lse[b] = res[b]
+    return out, lse
+
+
 def check(out, lse, ref_out, ref_lse, what=""):
     """Element-wise comparison; -inf lse must match exactly (empty rows)."""
     err = np.abs(out - ref_out)

@@ -141,3 +141,66 @@ def test_binding_rejects_a_cache_that_does_not_match_its_format():
                      (torch.zeros((2, 64, 576), dtype=torch.bfloat16), "fp16")]:
         with pytest.raises(ValueError):
             mla._check_cache(bad, fmt)
+
+
+def test_noalloc_argument_validation(lib):
+    # Every host-side check returns before anything is enqueued; on this
+    # GPU-less host the fake pointers are never dereferenced.
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+    f = lib.mla_decode_fwd_noalloc
+
+    def call(**over):
+        a = dict(q=16, kv=16, fmt=0, nb=10, bt=16, mp=4, L=16, batch=2, s_q=1, h_q=16, scale=0.0417, causal=0,
+                 sched=16, ns=16, parts=74, out=16, lse=16)
+        a.update(over)
+        return f(a["q"], a["kv"], a["fmt"], a["nb"], a["bt"], a["mp"], a["L"], a["batch"], a["s_q"], a["h_q"],
+                 a["scale"], a["causal"], a["sched"], a["ns"], a["parts"], a["out"], a["lse"], None)
+
+    assert call(q=None) == INVALID
+    assert call(parts=0) == INVALID           # same code as mla_decode_fwd
+    assert call(q=8) == INVALID
+    assert call(scale=float("nan")) == INVALID
+    assert call(s_q=2, h_q=128) == UNSUPPORTED
+    assert call(batch=16384, h_q=128) == WORKSPACE   # beyond the static scratch
+
+
+def test_wait_timeout_knob(lib):
+    import mla_paged_kv_04_b200 as mla
+    default = 2_000_000_000
+    first = mla.mla_set_wait_timeout_ns(5)
+    assert first == default
+    assert mla.mla_set_wait_timeout_ns(0) == 5        # 0 restores the default
+    assert mla.mla_set_wait_timeout_ns(0) == default
+
+
+def test_diagnostic_hooks_on_the_product_library(lib):
+    import mla_paged_kv_04_b200 as mla
+    UNSUPPORTED, INVALID = 2, 1
+    assert lib.mla_debug_trace_bytes() == 4 * 7 * 128 * 16 * 8
+    assert lib.mla_debug_set_trace_buffer(16, 1 << 20) == UNSUPPORTED   # records only in the trace build
+    assert lib.mla_debug_hold_at_tile(2, 3) == INVALID                 # misaligned flag
+    assert lib.mla_debug_hold_at_tile(None, -1) == 0
+    assert mla.mla_debug_trace_bytes() == 4 * 7 * 128 * 16 * 8
+
+
+def test_binding_rejects_host_tensors_before_the_c_abi():
+    import torch
+    import mla_paged_kv_04_b200 as mla
+    B = 2
+    q = torch.zeros((B, 1, 16, 576), dtype=torch.bfloat16)
+    kv = torch.zeros((3, 64, 576), dtype=torch.bfloat16)
+    bt = torch.zeros((B, 1), dtype=torch.int32)
+    L = torch.ones(B, dtype=torch.int32)
+    sched = torch.zeros(mla.mla_metadata_size(B, 74) // 4, dtype=torch.int32)
+    ns = torch.zeros(B + 1, dtype=torch.int32)
+    out = torch.zeros((B, 1, 16, 512), dtype=torch.bfloat16)
+    lse = torch.zeros((B, 1, 16), dtype=torch.float32)
+    ws = torch.zeros(mla.mla_workspace_size(B, 1, 16, 74), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        mla.mla_decode_fwd(q, kv, "bf16", bt, L, 0.04, False, sched, ns, 74, out, lse, ws)
+    with pytest.raises(ValueError):
+        mla.mla_decode_fwd_noalloc(q, kv, "bf16", bt, L, 0.04, False, sched, ns, 74, out, lse)
+    with pytest.raises(ValueError):
+        mla.mla_kv_append(torch.zeros((B, 1, 576), dtype=torch.bfloat16), kv, "bf16", bt, L, ws)
+    with pytest.raises(ValueError):
+        mla.mla_get_metadata(L, 1, 16, 74)
