@@ -21,6 +21,10 @@ Parity status per function (what pins it, see tests/test_oracle.py):
   gather_keys                         block-permutation invariance, poison
   mla_decode                          brute force, SDPA (library), closed forms
   mla_decode_partial + combine_splits split == unsplit, closed forms
+  mla_sparse_decode                   the full index list equals the dense
+                                      decode; permutation and padding
+                                      invariance; duplicate and single-key
+                                      closed forms; brute force
   encode_e4m3_rne                     every code round-trips, midpoints go to the
                                       even code, saturation; library cross-check
   quantize_fp8_656 / append_tokens    library cross-check of the codes, error
@@ -44,6 +48,7 @@ from .mla import (  # noqa: F401
     mla_decode_partial,
     combine_splits,
     mla_decode_rows,
+    mla_sparse_decode,
     encode_e4m3_rne,
     quantize_fp8_656,
     append_tokens,

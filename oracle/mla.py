@@ -258,6 +258,46 @@ def mla_decode(q_bits: np.ndarray, kv_cache: np.ndarray, fmt: str, block_table: 
     return out, lse
 
 
+def mla_sparse_decode(q_bits: np.ndarray, kv_cache: np.ndarray, fmt: str, block_table: np.ndarray,
+                      cache_seqlens: np.ndarray, indices: np.ndarray, softmax_scale: float):
+    """Sparse MLA decode: every query token attends only to its listed tokens.
+
+    The menfem.com DeepSeek page ("Key Contributions") names a sparse decode
+    kernel over the same 656-byte FP8 cache without defining it.  Reading R11:
+      indices int32 [b, s_q, topk] holds, for query token i of request b, the
+      positions j (0 <= j < L_b, the same positions the dense decode reads
+      through block_table) of the keys it attends to.  Entries outside
+      [0, L_b) are padding and are not keys.  Every valid entry is one term of
+      the softmax, so a position listed twice counts twice.  No causal mask:
+      the list alone decides what is visible.  A row with no valid entry gets
+      out = 0 and lse = -inf (R3).
+    For each head h:  x_k = softmax_scale * q[b,i,h] . K_{idx_k};
+      lse = ln sum_k e^{x_k};  out = sum_k e^{x_k - lse} K_{idx_k}[:512].
+    Returns out float64 [b, s_q, h_q, 512] and lse float64 [b, s_q, h_q].
+    """
+    B, s_q, h_q, d = q_bits.shape
+    assert d == D_QK
+    idx = np.asarray(indices, dtype=np.int64)
+    assert idx.shape[:2] == (B, s_q)
+    out = np.zeros((B, s_q, h_q, D_V))
+    lse = np.full((B, s_q, h_q), -np.inf)
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        keys = gather_keys(kv_cache, fmt, block_table[b], L)  # [L, 576]
+        q = decode_bf16_bits(q_bits[b])  # [s_q, h_q, 576]
+        for i in range(s_q):
+            sel = idx[b, i]
+            sel = sel[(sel >= 0) & (sel < L)]
+            if sel.size == 0:
+                continue
+            k = keys[sel]  # [n, 576], duplicates kept
+            x = softmax_scale * (q[i] @ k.T)  # [h_q, n]
+            lse_i, w = _softmax_rows(x)
+            lse[b, i] = lse_i
+            out[b, i] = w @ k[:, :D_V]
+    return out, lse
+
+
 def default_softmax_scale() -> float:
     """576^-0.5, the scale every configured workload uses."""
     return 1.0 / math.sqrt(D_QK)
