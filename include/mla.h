@@ -39,8 +39,12 @@
  *     that exceeded its time limit) are recorded in a status word inside the
  *     workspace; the first error recorded is kept until cleared.
  *   - Supported shapes: d_qk 576, d_v 512, one latent KV head, 64-token
- *     blocks, M = s_q * h_q rows per request with 1 <= M <= 128, bf16 q/out,
- *     fp32 lse; q, kv_cache and out 16-byte aligned; batch <= 16384.
+ *     blocks, M = s_q * h_q query rows per request with 1 <= M <= 1024, bf16
+ *     q/out, fp32 lse; q, kv_cache and out 16-byte aligned;
+ *     batch * ceil(M / 128) <= 16384.  A request with M > 128 is served as
+ *     ceil(M / 128) row tiles of at most 128 rows, scheduled like separate
+ *     requests that read the same pages (at about the same time, so that
+ *     the second read of a page is likely to come from L2).
  */
 #ifndef MLA_B200_H_
 #define MLA_B200_H_
@@ -72,8 +76,13 @@ const char* mla_status_string(mla_status_t status);
  * be queried. */
 int mla_default_num_sm_parts(int device);
 
-/* Bytes of the int32 schedule buffer `sched` for mla_get_metadata. */
-size_t mla_metadata_size(int batch, int num_sm_parts);
+/* Bytes of the int32 schedule buffer `sched` for mla_get_metadata (0 for a
+ * shape outside the supported set). */
+size_t mla_metadata_size(int batch, int s_q, int h_q, int num_sm_parts);
+
+/* Entries of the int32 `num_splits` array: batch * ceil(s_q * h_q / 128) + 1
+ * (0 for a shape outside the supported set). */
+int mla_num_splits_len(int batch, int s_q, int h_q);
 
 /*
  * Split-KV schedule (the split-KV idea follows from "optimized for
@@ -86,14 +95,17 @@ size_t mla_metadata_size(int batch, int num_sm_parts);
  * and nothing is split (no partial outputs, no combine work).
  *
  *   cache_seqlens  device int32 [batch], each >= 0
- *   s_q, h_q       query tokens and heads per request (only validated here)
+ *   s_q, h_q       query tokens and heads per request: they fix the row
+ *                  tiles per request, R = ceil(s_q * h_q / 128)
  *   num_sm_parts   CTA pairs the decode launch will use (>= 1)
  *   sched          device int32 buffer of mla_metadata_size() bytes (output)
- *   num_splits     device int32 [batch + 1] (output): exclusive prefix sum of
- *                  the number of splits per request; request b has
- *                  num_splits[b+1] - num_splits[b] splits.
+ *   num_splits     device int32 [batch * R + 1] (output): exclusive prefix
+ *                  sum of the number of splits per row tile; row tile t of
+ *                  request b (v = b * R + t) has num_splits[v+1] -
+ *                  num_splits[v] splits.
  * The same `sched`/`num_splits` are valid for any decode call with the same
- * cache_seqlens and num_sm_parts.  One tiny kernel, enqueued on `stream`.
+ * cache_seqlens, s_q * h_q row tiling and num_sm_parts.  One tiny kernel,
+ * enqueued on `stream`.
  */
 mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, int h_q,
                               int num_sm_parts, int32_t* sched, int32_t* num_splits,

@@ -62,7 +62,9 @@ def load_library(trace: bool = False):
     lib.mla_default_num_sm_parts.restype = c_int
     lib.mla_default_num_sm_parts.argtypes = [c_int]
     lib.mla_metadata_size.restype = c_size
-    lib.mla_metadata_size.argtypes = [c_int, c_int]
+    lib.mla_metadata_size.argtypes = [c_int, c_int, c_int, c_int]
+    lib.mla_num_splits_len.restype = c_int
+    lib.mla_num_splits_len.argtypes = [c_int, c_int, c_int]
     lib.mla_get_metadata.restype = c_int
     lib.mla_get_metadata.argtypes = [vp, c_int, c_int, c_int, c_int, vp, vp, vp]
     lib.mla_workspace_size.restype = c_size
@@ -154,10 +156,11 @@ def _check_decode_tensors(q, kv_cache, fmt, block_table, cache_seqlens, sched, n
         raise ValueError(f"out must be bf16 {(B, s_q, h_q, 512)}, got {out.dtype} {tuple(out.shape)}")
     if lse.shape != (B, s_q, h_q) or lse.dtype != torch.float32:
         raise ValueError(f"lse must be fp32 {(B, s_q, h_q)}, got {lse.dtype} {tuple(lse.shape)}")
-    if sched.dtype != torch.int32 or _nbytes(sched) < mla_metadata_size(B, int(num_sm_parts)):
-        raise ValueError(f"sched must be int32 of >= mla_metadata_size({B}, {num_sm_parts}) bytes")
-    if num_splits.dtype != torch.int32 or num_splits.numel() < B + 1:
-        raise ValueError(f"num_splits must be int32 [>= {B + 1}]")
+    if sched.dtype != torch.int32 or _nbytes(sched) < mla_metadata_size(B, s_q, h_q, int(num_sm_parts)):
+        raise ValueError(f"sched must be int32 of >= mla_metadata_size({B}, {s_q}, {h_q}, {num_sm_parts}) bytes")
+    n_len = mla_num_splits_len(B, s_q, h_q)
+    if num_splits.dtype != torch.int32 or num_splits.numel() < n_len:
+        raise ValueError(f"num_splits must be int32 [>= {n_len}]")
 
 
 def _check_cache(kv_cache: torch.Tensor, fmt: str):
@@ -185,8 +188,12 @@ def mla_default_num_sm_parts(device=None) -> int:
     return n
 
 
-def mla_metadata_size(batch: int, num_sm_parts: int) -> int:
-    return _active_lib().mla_metadata_size(batch, num_sm_parts)
+def mla_metadata_size(batch: int, s_q: int, h_q: int, num_sm_parts: int) -> int:
+    return _active_lib().mla_metadata_size(batch, s_q, h_q, num_sm_parts)
+
+
+def mla_num_splits_len(batch: int, s_q: int, h_q: int) -> int:
+    return _active_lib().mla_num_splits_len(batch, s_q, h_q)
 
 
 def mla_workspace_size(batch: int, s_q: int, h_q: int, num_sm_parts: int) -> int:
@@ -201,14 +208,17 @@ def mla_get_metadata(cache_seqlens: torch.Tensor, s_q: int, h_q: int, num_sm_par
         raise ValueError("cache_seqlens must be a CUDA int32 tensor")
     batch = cache_seqlens.numel()
     parts = mla_default_num_sm_parts(cache_seqlens.device) if num_sm_parts is None else int(num_sm_parts)
-    nbytes = lib.mla_metadata_size(batch, parts)
+    nbytes = lib.mla_metadata_size(batch, s_q, h_q, parts)
+    n_len = lib.mla_num_splits_len(batch, s_q, h_q)
+    if nbytes == 0 or n_len == 0:
+        raise MLAError(2, "mla_get_metadata")
     if sched is None:
         sched = torch.empty(max(nbytes // 4, 1), dtype=torch.int32, device=cache_seqlens.device)
     if num_splits is None:
-        num_splits = torch.empty(batch + 1, dtype=torch.int32, device=cache_seqlens.device)
+        num_splits = torch.empty(n_len, dtype=torch.int32, device=cache_seqlens.device)
     _on_device(cache_seqlens.device, cache_seqlens=cache_seqlens, sched=sched, num_splits=num_splits)
-    if sched.dtype != torch.int32 or num_splits.dtype != torch.int32 or num_splits.numel() < batch + 1:
-        raise ValueError(f"sched and num_splits must be int32, num_splits of >= {batch + 1} entries")
+    if sched.dtype != torch.int32 or num_splits.dtype != torch.int32 or num_splits.numel() < n_len:
+        raise ValueError(f"sched and num_splits must be int32, num_splits of >= {n_len} entries")
     if _nbytes(sched) < nbytes:
         raise MLAError(3, "mla_get_metadata")
     _check(lib.mla_get_metadata(cache_seqlens.data_ptr(), batch, s_q, h_q, parts, sched.data_ptr(),

@@ -16,8 +16,8 @@
 #include "entry.cuh"
 
 namespace mla {
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int parts, int32_t* sched, int32_t* num_splits,
-                            cudaStream_t stream);
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int rtiles, int parts, int32_t* sched,
+                            int32_t* num_splits, cudaStream_t stream);
 int metadata_max_batch();
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream);
 cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
@@ -79,10 +79,14 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// batch >= 1, s_q >= 1, h_q >= 1; M = s_q * h_q <= 128 * kMaxRowTiles and
+// batch * row_tiles(M) <= the schedule's batch limit.
 mla_status_t check_shape(int batch, int s_q, int h_q) {
   if (batch < 1 || s_q < 1 || h_q < 1) return MLA_ERR_INVALID_ARG;
-  if (batch > metadata_max_batch()) return MLA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(s_q) * h_q > kRows) return MLA_ERR_UNSUPPORTED;
+  const long long M = static_cast<long long>(s_q) * h_q;
+  if (M > static_cast<long long>(kRows) * kMaxRowTiles) return MLA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(batch) * row_tiles(static_cast<int>(M)) > metadata_max_batch())
+    return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
 
@@ -128,9 +132,14 @@ int mla_default_num_sm_parts(int device) {
   return sms / 2;
 }
 
-size_t mla_metadata_size(int batch, int num_sm_parts) {
-  if (batch < 1 || num_sm_parts < 1) return 0;
-  return sched_ints(batch, num_sm_parts) * sizeof(int32_t);
+int mla_num_splits_len(int batch, int s_q, int h_q) {
+  if (check_shape(batch, s_q, h_q) != MLA_OK) return 0;
+  return batch * row_tiles(s_q * h_q) + 1;
+}
+
+size_t mla_metadata_size(int batch, int s_q, int h_q, int num_sm_parts) {
+  if (check_shape(batch, s_q, h_q) != MLA_OK || num_sm_parts < 1) return 0;
+  return sched_ints(batch * row_tiles(s_q * h_q), num_sm_parts) * sizeof(int32_t);
 }
 
 mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int num_sm_parts,
@@ -140,7 +149,8 @@ mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, 
   if (num_sm_parts < 1 || num_sm_parts > 65535) return MLA_ERR_INVALID_ARG;
   mla_status_t st = check_shape(batch, s_q, h_q);
   if (st != MLA_OK) return st;
-  cudaError_t e = launch_metadata(cache_seqlens, batch, num_sm_parts, sched, num_splits,
+  const int rt = row_tiles(s_q * h_q);
+  cudaError_t e = launch_metadata(cache_seqlens, batch * rt, rt, num_sm_parts, sched, num_splits,
                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -200,6 +210,7 @@ mla_status_t launch_decode_call(const void* q, const void* kv_cache, mla_kv_form
   p.s_q = s_q;
   p.h_q = h_q;
   p.M = M;
+  p.row_tiles = row_tiles(M);
   p.causal = causal ? 1 : 0;
   p.num_parts = num_sm_parts;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
@@ -243,6 +254,7 @@ mla_status_t launch_decode_call(const void* q, const void* kv_cache, mla_kv_form
   c.lse = lse;
   c.batch = batch;
   c.M = M;
+  c.row_tiles = row_tiles(M);
   c.num_parts = num_sm_parts;
   e = launch_combine(c, num_sm_parts, s);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;

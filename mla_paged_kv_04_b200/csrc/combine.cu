@@ -16,7 +16,7 @@ namespace mla {
 constexpr int kCombineWarps = 4;  // one query row per warp
 constexpr int kCombineUnroll = 4;  // splits whose partial rows are in flight at once
 
-// grid.x walks the schedule's list of split requests (at most one per CTA
+// grid.x walks the schedule's list of split (virtual) requests (at most one per CTA
 // pair), grid.y covers the query rows four at a time, one row per warp.  Lane
 // s holds split s's weight (in chunks of 32 splits); the partial rows of
 // kCombineUnroll splits are loaded together so that their latencies overlap.
@@ -24,19 +24,21 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
   pdl_wait();  // the decode kernel has completed
   // a schedule made for another CTA-pair count or batch: reported by the
   // decode kernel, nothing to merge
-  if (p.sched[0] != p.num_parts || p.sched[3] != p.batch) return;
+  if (p.sched[0] != p.num_parts || p.sched[3] != p.batch * p.row_tiles || p.sched[7] != p.row_tiles) return;
   const int num_split_req = p.sched[5];
   if (static_cast<int>(blockIdx.x) >= num_split_req) return;
   const int parts = p.sched[0];
-  const int b = p.sched[sched_split_list_offset(parts) + blockIdx.x];
-  const int first = p.num_splits[b];
-  const int nsplit = p.num_splits[b + 1] - first;
+  const int vb = p.sched[sched_split_list_offset(parts) + blockIdx.x];  // virtual request
+  const int b = vb / p.row_tiles, row0 = (vb - b * p.row_tiles) * kRows;
+  const int mt = rows_per_tile(p.M);  // partial rows per slot
+  const int first = p.num_splits[vb];
+  const int nsplit = p.num_splits[vb + 1] - first;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y * kCombineWarps + warp;
-  if (r >= p.M) return;
+  const int r = blockIdx.y * kCombineWarps + warp;  // row within the row tile
+  if (r >= mt || row0 + r >= p.M) return;
 
   float m = -CUDART_INF_F;
-  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, p.lse_part[static_cast<size_t>(first + s) * p.M + r]);
+  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, p.lse_part[static_cast<size_t>(first + s) * mt + r]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
 
@@ -48,7 +50,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
     for (int s0 = 0; s0 < nsplit; s0 += 32) {
       float w = 0.f;
       if (s0 + lane < nsplit) {
-        const float ls = p.lse_part[static_cast<size_t>(first + s0 + lane) * p.M + r];
+        const float ls = p.lse_part[static_cast<size_t>(first + s0 + lane) * mt + r];
         w = (ls == -CUDART_INF_F) ? 0.f : expf(ls - m);
       }
       wsum += w;
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
           wk[u] = __shfl_sync(0xffffffffu, w, (k + u) & 31);
           if (k + u >= cnt) wk[u] = 0.f;
           const float4* src =
-              reinterpret_cast<const float4*>(p.o_part + (static_cast<size_t>(first + s0 + k + u) * p.M + r) * kDv) +
+              reinterpret_cast<const float4*>(p.o_part + (static_cast<size_t>(first + s0 + k + u) * mt + r) * kDv) +
               lane * 4;
 #pragma unroll
           for (int v = 0; v < 4; ++v) x[u][v] = wk[u] != 0.f ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -89,15 +91,16 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r2) : "f"(acc[2 * i + 1] * inv), "f"(acc[2 * i] * inv));
     packed[i] = r2;
   }
-  uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(b) * p.M + r) * kDv + lane * 16);
+  const size_t orow = static_cast<size_t>(b) * p.M + row0 + r;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + lane * 16);
   dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-  if (lane == 0) p.lse[static_cast<size_t>(b) * p.M + r] = wsum > 0.f ? m + logf(wsum) : -CUDART_INF_F;
+  if (lane == 0) p.lse[orow] = wsum > 0.f ? m + logf(wsum) : -CUDART_INF_F;
 }
 
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(parts, (p.M + kCombineWarps - 1) / kCombineWarps);
+  cfg.gridDim = dim3(parts, (rows_per_tile(p.M) + kCombineWarps - 1) / kCombineWarps);
   cfg.blockDim = dim3(32 * kCombineWarps);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -13,6 +13,16 @@ constexpr int kDqk = 576;         // key width: 512 latent + 64 RoPE
 constexpr int kDv = 512;          // value width (the latent)
 constexpr int kDRope = 64;
 constexpr int kRows = 128;        // MMA M: query rows (s_q * h_q, padded) per work item
+constexpr int kMaxRowTiles = 8;   // M = s_q * h_q <= 1024: up to 8 row tiles per request
+
+// A request with M = s_q * h_q query rows is served as ceil(M / 128) row
+// tiles; the schedule treats every (request, row tile) as a unit of its own
+// ("virtual request" v = request * row_tiles + tile), so the tiles of one
+// request run on different CTA pairs at about the same time and share its
+// pages through L2.
+__host__ __device__ inline int row_tiles(int M) { return (M + kRows - 1) / kRows; }
+// Rows of a row tile's partial results in the workspace (the stride per slot).
+__host__ __device__ inline int rows_per_tile(int M) { return M < kRows ? M : kRows; }
 constexpr int kFp8TokenBytes = 656;
 
 // Per-request fixed cost of the split-KV schedule, in units of one page.
@@ -28,10 +38,11 @@ constexpr int kSplitOverheadPages = 4;
 // cut by more than this many pages.
 constexpr int kSplitPenaltyPages = 16;
 
-// Schedule buffer (int32) written by the metadata kernel:
-//   [0] num_parts  [1] total_items  [2] units per part  [3] batch
-//   [4] overhead   [5] number of split requests  [6] 1 if whole requests
-//   (one per part, no split), else 0   [7] reserved
+// Schedule buffer (int32) written by the metadata kernel, over the virtual
+// requests (request, row tile) of the batch:
+//   [0] num_parts  [1] total_items  [2] units per part  [3] virtual batch
+//   (batch * row tiles)  [4] overhead   [5] number of split virtual requests
+//   [6] 1 if whole requests (one per part, no split), else 0  [7] row tiles
 //   [8, 8 + num_parts + 1)          first item index of each part
 //   then num_parts ints             ids of the split requests (first [5] valid)
 //   then (16-byte aligned) 4 ints per item: request b, first page, end page, slot
@@ -49,16 +60,19 @@ __host__ __device__ inline size_t sched_ints(int batch, int parts) {
 __host__ __device__ inline int max_items(int batch, int parts) { return batch + parts; }
 
 // Workspace: a 256-byte header (status word at offset 0), then fp32 partial
-// lse [max_items][M] and fp32 partial outputs [max_items][M][512].
+// lse [max_items][Mt] and fp32 partial outputs [max_items][Mt][512], with
+// max_items over the virtual batch and Mt = rows_per_tile(M).
 constexpr size_t kWsHeader = 256;
 __host__ __device__ inline size_t ws_lse_offset() { return kWsHeader; }
 __host__ __device__ inline size_t ws_o_offset(int batch, int parts, int M) {
-  size_t lse_bytes = 4ull * static_cast<size_t>(max_items(batch, parts)) * static_cast<size_t>(M);
+  const int vb = batch * row_tiles(M);
+  size_t lse_bytes = 4ull * static_cast<size_t>(max_items(vb, parts)) * static_cast<size_t>(rows_per_tile(M));
   return kWsHeader + ((lse_bytes + 255) / 256) * 256;
 }
 __host__ __device__ inline size_t ws_bytes(int batch, int parts, int M) {
+  const int vb = batch * row_tiles(M);
   return ws_o_offset(batch, parts, M) +
-         4ull * static_cast<size_t>(max_items(batch, parts)) * static_cast<size_t>(M) * kDv;
+         4ull * static_cast<size_t>(max_items(vb, parts)) * static_cast<size_t>(rows_per_tile(M)) * kDv;
 }
 
 struct DecodeParams {
@@ -76,7 +90,8 @@ struct DecodeParams {
   int batch;
   int s_q;
   int h_q;
-  int M;
+  int M;                        // query rows per request (s_q * h_q)
+  int row_tiles;                // ceil(M / 128)
   int causal;
   int num_parts;                // CTA pairs launched (must equal sched[0])
   float scale_log2;             // softmax_scale * log2(e)
@@ -119,6 +134,7 @@ struct CombineParams {
   float* lse;
   int batch;
   int M;
+  int row_tiles;
   int num_parts;
 };
 

@@ -76,12 +76,26 @@ constexpr int kXBufBytes = kXMsgBytes;
 // has read tile g's (a remote arrive on the peer's "buffer free" barrier).
 constexpr int kXBuffers = 2;
 constexpr int kSoftmaxWarps = 8;
+// FP8: one dequant warp per scheduler partition (a warpgroup).
+constexpr int kDqWarps = 4;
+// FP8 register split per warpgroup (512 threads launch with 128 registers
+// each): control 64, softmax 176, dequant 96, and the softmax and dequant
+// warpgroups at 64 for the common tail.  64 + 2 x 176 + 96 = 4 x 128: the
+// softmax warpgroups' increase is exactly funded by the decreases.  (ptxas
+// does not fit the dequant warpgroup's code below 96 registers.)
+constexpr int kRegLaunchFp8 = 128;
+constexpr int kRegCtl = 64;
+constexpr int kRegSoftmax = 176;
+constexpr int kRegDq = 96;
+constexpr int kRegTail = 64;
+static_assert(kRegCtl + 2 * kRegSoftmax + (kDqWarps / 4) * kRegDq <= (3 + kDqWarps / 4) * kRegLaunchFp8,
+              "register split exceeds the launch budget");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: the lazy reference moves by more than a factor 256
 
 template <bool kFp8>
 struct Cfg {
   static constexpr int kStages = kFp8 ? 3 : 5;  // bf16 page-half stages
-  static constexpr int kThreads = kFp8 ? 512 : 384;
+  static constexpr int kThreads = kFp8 ? 384 + 32 * kDqWarps : 384;
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kFull + kStages;
   static constexpr int kSFull = kEmpty + kStages;  // two: by tile parity
@@ -233,7 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(BAR(C::kFull + i), kFp8 ? 4 : 1);  // FP8: the four dequant warps arrive
+      mbar_init(BAR(C::kFull + i), kFp8 ? kDqWarps : 1);  // FP8: every dequant warp arrives
       mbar_init(BAR(C::kEmpty + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -250,7 +264,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
-      mbar_init(BAR(C::kRawEmpty + i), 4);
+      mbar_init(BAR(C::kRawEmpty + i), kDqWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -294,7 +308,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   const int num_parts = p.sched[0];
   const int32_t* items = p.sched + sched_items_offset(num_parts);
   int it_begin = 0, it_end = 0;
-  if (num_parts != p.num_parts || p.sched[3] != p.batch) {
+  if (num_parts != p.num_parts || p.sched[3] != p.batch * p.row_tiles || p.sched[7] != p.row_tiles) {
     // schedule made for another CTA-pair count or another batch: its request
     // ids and item slots may lie outside this call's tensors and workspace,
     // so do nothing and report it
@@ -304,16 +318,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     it_end = p.sched[kSchedHeader + part + 1];
   }
 
-  // Register budget per warpgroup.  FP8 launches 512 threads with 128
-  // registers each (65,536 in all) and moves them to the softmax warpgroups:
-  // 64 + 2 x 176 + 96 = 4 x 128.  The only increase is the softmax
-  // warpgroups' at their start, which the two decreases exactly fund; at the
-  // end every warpgroup decreases to 64 for the short common tail.  (An
-  // increase anywhere else could take registers that a softmax warpgroup
-  // still waits for: setmaxnreg.inc blocks until the pool can pay.)
-  static_assert(64 + 2 * 176 + 96 <= 4 * 128, "register split exceeds the launch budget");
+  // Register budget per warpgroup (FP8, constants above).  The only increase
+  // is the softmax warpgroups' at their start, which the decreases exactly
+  // fund; at the end every warpgroup is at kRegTail for the short common
+  // tail.  (An increase anywhere else could take registers that a softmax
+  // warpgroup still waits for: setmaxnreg.inc blocks until the pool can pay.)
   if (warp < 4) {
-    if constexpr (kFp8) setmaxnreg_dec<64>();
+    if constexpr (kFp8) setmaxnreg_dec<kRegCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -325,15 +336,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       uint32_t g = 0;
       bool ok = true;
       for (int it = it_begin; it < it_end && ok; ++it) {
-        const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
+        const int vb = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
+        const int b = vb / p.row_tiles, row0 = (vb - b * p.row_tiles) * kRows;
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
         // This producer runs kStages pages ahead: start this item's Q rows
         // towards L2 now, so that the softmax warps' Q loads at the item
         // boundary do not wait on DRAM behind the page stream (rank 0 fetches
         // whole rows for both CTAs; q rows are contiguous, 1152 B each).
         if (rank == 0 && p1 > p0) {
-          const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q) + static_cast<size_t>(b) * p.M * (kDqk * 2);
-          const uint32_t bytes = static_cast<uint32_t>(p.M) * (kDqk * 2);
+          const uint8_t* qb =
+              reinterpret_cast<const uint8_t*>(p.q) + (static_cast<size_t>(b) * p.M + row0) * (kDqk * 2);
+          const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.M - row0)) * (kDqk * 2);
           for (uint32_t o = 0; o < bytes; o += 16384u) prefetch_l2_bulk(qb + o, min(16384u, bytes - o));
         }
         for (int pg = p0; pg < p1; ++pg, ++g) {
@@ -449,9 +462,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       mbar_wait(BAR(C::kDrain + 1), 0, &g_never_abort, 100000000ull);
     }
   }
+    __syncwarp();
+    static_assert(kRegCtl == kRegTail, "the control warps stay at their budget for the tail");
   } else if (warp < 4 + kSoftmaxWarps) {
     // ------------------------------------------------------------------ softmax / epilogue
-    if constexpr (kFp8) setmaxnreg_inc<176>();
+    if constexpr (kFp8) setmaxnreg_inc<kRegSoftmax>();
     const int wg = (warp - 4) >> 2;         // warpgroup: the tiles g with g % 2 == wg
     const int wq = warp & 3;                // tensor-memory lane quarter
     const int r = wq * 32 + lane;           // query row == tensor-memory lane
@@ -471,17 +486,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     uint32_t g = 0;      // tile counter of this CTA (every tile, both warpgroups)
     uint32_t nitem = 0;  // items with at least one page
     bool ok = true;
-    const bool row_ok = r < p.M;
-    const int qi = r / p.h_q;
+    const int mt = rows_per_tile(p.M);  // partial-result rows per slot
     for (int it = it_begin; it < it_end && ok; ++it) {
-      const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2], slot = items[4 * it + 3];
+      const int vb = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2], slot = items[4 * it + 3];
+      const int b = vb / p.row_tiles, row0 = (vb - b * p.row_tiles) * kRows;
+      const bool row_ok = row0 + r < p.M;   // this thread's row exists in the request
+      const int qi = (row0 + r) / p.h_q;    // its query token
       const int L = p.seqlens[b];
       const int n = p1 - p0;
-      const size_t orow = static_cast<size_t>(b) * p.M + r;
+      const size_t orow = static_cast<size_t>(b) * p.M + row0 + r;
       if (n <= 0) {
         if (row_ok) {
           if (slot >= 0) {
-            if (rank == 0 && wg == 0) p.lse_part[static_cast<size_t>(slot) * p.M + r] = -CUDART_INF_F;
+            if (rank == 0 && wg == 0) p.lse_part[static_cast<size_t>(slot) * mt + r] = -CUDART_INF_F;
           } else {
             uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256 + wg * 128);
             for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
@@ -769,7 +786,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
                                   pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(slot) * p.M + r) * kDv +
+            float4* dst = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(slot) * mt + r) * kDv +
                                                     rank * 256 + col);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
@@ -780,25 +797,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       }
       if (row_ok && rank == 0 && wg == 0) {
         if (slot < 0) p.lse[orow] = lse_val;
-        else p.lse_part[static_cast<size_t>(slot) * p.M + r] = lse_val;
+        else p.lse_part[static_cast<size_t>(slot) * mt + r] = lse_val;
       }
       if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 3);
     }
     if (!ok) raise_abort(p, abort_flag);
     __syncwarp();
-    if constexpr (kFp8) setmaxnreg_dec<64>();
+    if constexpr (kFp8) setmaxnreg_dec<kRegTail>();
   } else if (kFp8) {
     // ------------------------------------------------------------------ FP8 dequant (warps 12-15)
-    setmaxnreg_dec<96>();
+    setmaxnreg_dec<kRegDq>();
     // Raw 656-byte tokens -> this CTA's bf16 page half, in the same swizzled
     // layout the BF16 path gets from TMA.  Thread dt handles 16-code units
     // u = dt + 128 k: token u / 16, codes 16 (u % 16) .. +16 of the CTA's 256.
+    constexpr int kDqThreads = 32 * kDqWarps;
     const int dt = threadIdx.x - 128 - kSoftmaxWarps * 32;
     uint32_t g = 0;
     bool ok = true;
     for (int it = it_begin; it < it_end && ok; ++it) {
-      const int b = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
-      const int L = p.seqlens[b];
+      const int p0 = items[4 * it + 1], p1 = items[4 * it + 2];
+      const int L = p.seqlens[items[4 * it] / p.row_tiles];
       const int last_page = (L - 1) / kPage;
       for (int pg = p0; pg < p1; ++pg, ++g) {
         const uint32_t rs = g % kRawStages, st = g % kStages;
@@ -814,8 +832,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const uint8_t* rrope = rscale + kRawScaleBytes;
         uint8_t* dst = sbase + st * kStageBytes;
 #pragma unroll 2
-        for (int k = 0; k < 8; ++k) {
-          const int u = dt + 128 * k;
+        for (int k = 0; k < 1024 / kDqThreads; ++k) {
+          const int u = dt + kDqThreads * k;
           const int t = u >> 4, g16 = u & 15;
           uint32_t w[8];
           if (t < valid) {
@@ -832,8 +850,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           *reinterpret_cast<uint4*>(row + (((u0 + 1) ^ (t & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
         }
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int u = dt + 128 * k;
+        for (int k = 0; k < 256 / kDqThreads; ++k) {
+          const int u = dt + kDqThreads * k;
           const int t = u >> 2, w4 = u & 3;
           uint4 v = make_uint4(0, 0, 0, 0);
           if (t < valid) v = *reinterpret_cast<const uint4*>(rrope + t * 64 + w4 * 16);
@@ -850,7 +868,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
     if (!ok) raise_abort(p, abort_flag);
     __syncwarp();
-    setmaxnreg_dec<64>();
+    setmaxnreg_dec<kRegTail>();
   }
 
   tc_fence_before();

@@ -6,9 +6,14 @@ implementation the device kernel is tested against.  `validate` checks the
 invariants every schedule must satisfy; `parse` turns the int32 buffer into
 per-part work lists.
 
+Requests with M = s_q * h_q > 128 query rows are planned as ceil(M / 128)
+row tiles, each a "virtual request" v = b * row_tiles + tile with request b's
+length; everything below (items, splits, num_splits) is over virtual requests.
+
 Buffer layout (int32):
-  [0] parts [1] items [2] units per part [3] batch [4] per-request overhead
-  [5] split requests [6] 1 in whole-request mode [7] reserved
+  [0] parts [1] items [2] units per part [3] virtual batch [4] per-request
+  overhead [5] split (virtual) requests [6] 1 in whole-request mode
+  [7] row tiles
   [8, 8 + parts + 1)      first item of each part
   then `parts` ints       ids of split requests (first [5] valid)
   then, 16-byte aligned,  4 ints per item: request, first page, end page, slot
@@ -40,9 +45,14 @@ def sched_ints(batch: int, parts: int) -> int:
     return items_offset(parts) + 4 * (batch + parts)
 
 
-def plan(seqlens, parts: int, overhead: int = DEFAULT_OVERHEAD):
-    """Host computation of the schedule -> (sched int32[sched_ints], num_splits int32[batch+1])."""
-    L = np.maximum(np.asarray(seqlens, dtype=np.int64), 0)
+def row_tiles(s_q: int, h_q: int) -> int:
+    return -(-(s_q * h_q) // 128)
+
+
+def plan(seqlens, parts: int, overhead: int = DEFAULT_OVERHEAD, rtiles: int = 1):
+    """Host computation of the schedule -> (sched int32[sched_ints], num_splits
+    int32[batch * rtiles + 1]), over the virtual requests of `rtiles` row tiles."""
+    L = np.repeat(np.maximum(np.asarray(seqlens, dtype=np.int64), 0), rtiles)
     B = L.size
     n = (L + PAGE - 1) // PAGE
     cost = n + overhead
@@ -51,7 +61,7 @@ def plan(seqlens, parts: int, overhead: int = DEFAULT_OVERHEAD):
     t = max(1, -(-T // parts))
     if B <= parts and int(cost.max(initial=0)) <= t + SPLIT_PENALTY:
         sched = np.zeros(sched_ints(B, parts), dtype=np.int32)
-        sched[:8] = (parts, B, int(cost.max(initial=0)), B, overhead, 0, 1, 0)
+        sched[:8] = (parts, B, int(cost.max(initial=0)), B, overhead, 0, 1, rtiles)
         sched[HEADER:HEADER + parts + 1] = np.minimum(np.arange(parts + 1), B)
         io = items_offset(parts)
         items = np.stack([np.arange(B), np.zeros(B, dtype=np.int64), n, np.full(B, -1)], axis=1)
@@ -76,7 +86,7 @@ def plan(seqlens, parts: int, overhead: int = DEFAULT_OVERHEAD):
             items[idx] = (b, p0, p1, idx if K[b] > 1 else -1)
         if K[b] > 1:
             split_reqs.append(b)
-    sched[:8] = (parts, I, t, B, overhead, len(split_reqs), 0, 0)
+    sched[:8] = (parts, I, t, B, overhead, len(split_reqs), 0, rtiles)
     for k in range(parts + 1):
         pos = k * t
         if k == parts or pos >= T:
@@ -101,13 +111,15 @@ def parse(sched, parts: int):
     return [[tuple(int(x) for x in items[i]) for i in range(first[k], first[k + 1])] for k in range(parts)]
 
 
-def validate(sched, num_splits, seqlens, parts: int):
-    """Raise AssertionError unless the schedule is a valid split-KV plan for `seqlens`."""
+def validate(sched, num_splits, seqlens, parts: int, rtiles: int = 1):
+    """Raise AssertionError unless the schedule is a valid split-KV plan for
+    `seqlens` with `rtiles` row tiles per request (every page of every row
+    tile covered exactly once)."""
     sched = np.asarray(sched)
-    L = np.maximum(np.asarray(seqlens, dtype=np.int64), 0)
+    L = np.repeat(np.maximum(np.asarray(seqlens, dtype=np.int64), 0), rtiles)
     B = L.size
     n = (L + PAGE - 1) // PAGE
-    assert int(sched[0]) == parts and int(sched[3]) == B
+    assert int(sched[0]) == parts and int(sched[3]) == B and int(sched[7]) == rtiles
     I = int(sched[1])
     assert 0 < I <= B + parts
     first = sched[HEADER:HEADER + parts + 1]

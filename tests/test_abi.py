@@ -46,12 +46,20 @@ def test_status_strings(lib):
 def test_sizes(lib):
     import mla_paged_kv_04_b200 as mla
     from mla_paged_kv_04_b200 import schedule
-    assert mla.mla_metadata_size(64, 74) == 4 * schedule.sched_ints(64, 74)
-    assert mla.mla_metadata_size(0, 74) == 0
+    assert mla.mla_metadata_size(64, 1, 128, 74) == 4 * schedule.sched_ints(64, 74)
+    assert mla.mla_metadata_size(64, 2, 128, 74) == 4 * schedule.sched_ints(128, 74)   # two row tiles
+    assert mla.mla_metadata_size(0, 1, 128, 74) == 0
+    assert mla.mla_num_splits_len(64, 1, 128) == 65
+    assert mla.mla_num_splits_len(64, 3, 128) == 64 * 3 + 1
+    assert mla.mla_num_splits_len(64, 9, 128) == 0                                     # M = 1152 > 1024
     w1 = mla.mla_workspace_size(64, 1, 128, 74)
     w2 = mla.mla_workspace_size(64, 1, 128, 148)
     assert w1 >= 256 + (64 + 74) * 128 * 513 * 4 and w2 > w1
-    assert mla.mla_workspace_size(1, 2, 128, 74) == 0  # M = 256 unsupported
+    w3 = mla.mla_workspace_size(1, 2, 128, 74)      # M = 256: two row tiles of 128 rows
+    assert w3 >= 256 + (2 + 74) * 128 * 513 * 4
+    assert mla.mla_workspace_size(1, 8, 128, 74) > 0
+    assert mla.mla_workspace_size(1, 9, 128, 74) == 0  # M = 1152 > 1024 unsupported
+    assert mla.mla_workspace_size(4096, 8, 128, 74) == 0  # 32768 row tiles > 16384
 
 
 def _call_decode(lib, **over):
@@ -77,7 +85,8 @@ def test_decode_argument_validation(lib):
     assert _call_decode(lib, scale=float("nan")) == INVALID
     assert _call_decode(lib, scale=float("inf")) == INVALID
     assert _call_decode(lib, batch=0) == INVALID
-    assert _call_decode(lib, s_q=2, h_q=128) == UNSUPPORTED   # M = 256 > 128
+    assert _call_decode(lib, s_q=9, h_q=128) == UNSUPPORTED   # M = 1152 > 1024
+    assert _call_decode(lib, s_q=2, h_q=128, ws_bytes=1024) == WORKSPACE   # M = 256 is supported
     assert _call_decode(lib, batch=20000) == UNSUPPORTED
     assert _call_decode(lib, ws_bytes=1024) == WORKSPACE
 
@@ -116,7 +125,7 @@ def test_metadata_argument_validation(lib):
     assert f(16, 4, 1, 128, 0, 16, 16, None) == INVALID
     assert f(16, 4, 1, 128, 74, 8, 16, None) == INVALID   # sched must be 16-byte aligned
     assert f(16, 0, 1, 128, 74, 16, 16, None) == INVALID
-    assert f(16, 4, 3, 64, 74, 16, 16, None) == UNSUPPORTED
+    assert f(16, 4, 17, 64, 74, 16, 16, None) == UNSUPPORTED   # M = 1088 > 1024
 
 
 def test_product_has_no_oracle_dependency():
@@ -160,7 +169,7 @@ def test_noalloc_argument_validation(lib):
     assert call(parts=0) == INVALID           # same code as mla_decode_fwd
     assert call(q=8) == INVALID
     assert call(scale=float("nan")) == INVALID
-    assert call(s_q=2, h_q=128) == UNSUPPORTED
+    assert call(s_q=9, h_q=128) == UNSUPPORTED
     assert call(batch=16384, h_q=128) == WORKSPACE   # beyond the static scratch
 
 
@@ -191,7 +200,7 @@ def test_binding_rejects_host_tensors_before_the_c_abi():
     kv = torch.zeros((3, 64, 576), dtype=torch.bfloat16)
     bt = torch.zeros((B, 1), dtype=torch.int32)
     L = torch.ones(B, dtype=torch.int32)
-    sched = torch.zeros(mla.mla_metadata_size(B, 74) // 4, dtype=torch.int32)
+    sched = torch.zeros(mla.mla_metadata_size(B, 1, 16, 74) // 4, dtype=torch.int32)
     ns = torch.zeros(B + 1, dtype=torch.int32)
     out = torch.zeros((B, 1, 16, 512), dtype=torch.bfloat16)
     lse = torch.zeros((B, 1, 16), dtype=torch.float32)

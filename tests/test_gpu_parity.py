@@ -48,6 +48,17 @@ SMALL = [
     (2, 4, 32, (333, 4), True),       # s_q = 4
 ]
 
+# M = s_q * h_q above 128: row tiles of 128 rows scheduled as separate units
+WIDE = [
+    # batch, s_q, h_q, seqlens, causal, parts
+    (2, 2, 128, (700, 1500), True, None),     # M = 256, speculative pair with 128 heads
+    (3, 4, 64, (65, 2000, 3), True, None),    # M = 256
+    (1, 3, 128, (2500,), True, None),         # M = 384, three row tiles
+    (2, 2, 100, (900, 64), False, None),      # M = 200: a full and a partial row tile
+    (2, 8, 128, (1200, 130), True, None),     # M = 1024, the largest
+    (3, 2, 128, (3000, 100, 1777), True, 7),  # row tiles and split-KV together
+]
+
 
 @pytest.mark.parametrize("batch,s_q,h_q,seqlens,causal", SMALL)
 def test_small_bf16(batch, s_q, h_q, seqlens, causal):
@@ -56,6 +67,23 @@ def test_small_bf16(batch, s_q, h_q, seqlens, causal):
     assert st == 0
     ro, rl = oracle_for(c)
     check(out, lse, ro, rl, f"bf16 {seqlens}")
+
+
+@pytest.mark.parametrize("batch,s_q,h_q,seqlens,causal,parts", WIDE)
+def test_wide_rows_bf16(batch, s_q, h_q, seqlens, causal, parts):
+    c = _case(batch, s_q, h_q, seqlens, causal=causal, seed=40 + s_q * h_q)
+    out, lse, st = run_gpu(c, num_sm_parts=parts)
+    assert st == 0
+    ro, rl = oracle_for(c)
+    check(out, lse, ro, rl, f"bf16 M={s_q * h_q} {seqlens}")
+
+
+def test_wide_rows_fp8():
+    c = _case(2, 2, 128, (1500, 333), fmt="fp8_656", causal=True, seed=44)
+    out, lse, st = run_gpu(c)
+    assert st == 0
+    ro, rl = oracle_for(c, dequant_bf16=True)
+    check(out, lse, ro, rl, "fp8 M=256")
 
 
 @pytest.mark.parametrize("batch,s_q,h_q,seqlens,causal", SMALL[:4])
@@ -140,6 +168,21 @@ def test_metadata_covers_every_page_once():
         np.testing.assert_array_equal(dev_sched[:8], host_sched[:8])
         np.testing.assert_array_equal(dev_sched[8:8 + parts + 1], host_sched[8:8 + parts + 1])
         io = schedule.items_offset(parts)
+        np.testing.assert_array_equal(dev_sched[io:used], host_sched[io:used])
+    # two and three row tiles per request (M = 256, 384)
+    for s_q, rt in ((2, 2), (3, 3)):
+        L = torch.randint(0, 5000, (41,), generator=g, dtype=torch.int32)
+        sched, ns = mla.mla_get_metadata(L.cuda(), s_q, 128, 74)
+        torch.cuda.synchronize()
+        dev_sched, dev_ns = sched.cpu().numpy(), ns.cpu().numpy()
+        schedule.validate(dev_sched, dev_ns, L.numpy(), 74, rtiles=rt)
+        host_sched, host_ns = schedule.plan(L.numpy(), 74, rtiles=rt)
+        np.testing.assert_array_equal(dev_ns, host_ns)
+        np.testing.assert_array_equal(dev_sched[:8 + 74 + 1], host_sched[:8 + 74 + 1])
+        off, nsr = schedule.split_list_offset(74), int(host_sched[5])
+        np.testing.assert_array_equal(dev_sched[off:off + nsr], host_sched[off:off + nsr])
+        io = schedule.items_offset(74)
+        used = io + 4 * int(host_sched[1])
         np.testing.assert_array_equal(dev_sched[io:used], host_sched[io:used])
 
 

@@ -31,16 +31,20 @@ def _lib():
     mla.load_library()
 
 
-@pytest.mark.parametrize("fmt,parts", [("bf16", None), ("fp8_656", None), ("bf16", 8)])
+# Few CTA pairs, so that the pairs run past the held tile (with the default 74
+# pairs these requests would be cut into items of one or two pages).
+@pytest.mark.parametrize("fmt,parts", [("bf16", 2), ("fp8_656", 2), ("bf16", 4)])
 def test_wait_that_runs_out_is_reported_and_the_next_call_is_correct(fmt, parts):
     import mla_paged_kv_04_b200 as mla
+    from mla_paged_kv_04_b200 import schedule
     dev = torch.device("cuda")
     w = W.Workload("timeout", 3, 1, 128, (1, 1), fmt=fmt, seed=31)
     c = W.make_case(w, seqlens=[2000, 1500, 700])  # 32, 24 and 11 pages
     q, kv, bt, L = (c[k].to(dev) for k in ("q", "kv_cache", "block_table", "cache_seqlens"))
     B = 3
-    parts = parts or mla.mla_default_num_sm_parts()
     sched, ns = mla.mla_get_metadata(L, 1, 128, parts)
+    per_pair = [sum(p1 - p0 for _, p0, p1, _ in part) for part in schedule.parse(sched.cpu().numpy(), parts)]
+    assert max(per_pair) > 5, per_pair  # some pair reaches the held tile (one is enough to time out)
     ws = mla.alloc_workspace(B, 1, 128, parts, dev)
     out = torch.empty((B, 1, 128, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, 1, 128), dtype=torch.float32, device=dev)

@@ -75,3 +75,18 @@ def test_batch_above_parts_uses_the_balanced_cut():
     sched, ns = schedule.plan(L, 74)
     schedule.validate(sched, ns, L, 74)
     assert int(sched[6]) == 0
+
+
+@pytest.mark.parametrize("rtiles", [2, 3, 8])
+def test_row_tiles_are_planned_as_virtual_requests(rtiles):
+    rng = np.random.default_rng(rtiles)
+    for parts in (1, 5, 74):
+        L = rng.integers(0, 6000, 23)
+        sched, ns = schedule.plan(L, parts, rtiles=rtiles)
+        schedule.validate(sched, ns, L, parts, rtiles=rtiles)
+        assert int(sched[3]) == 23 * rtiles and int(sched[7]) == rtiles and ns.size == 23 * rtiles + 1
+        # every row tile of request b has request b's pages
+        items = [it for part in schedule.parse(sched, parts) for it in part]
+        for v in range(23 * rtiles):
+            pages = sum(p1 - p0 for vb, p0, p1, _ in items if vb == v)
+            assert pages == -(-int(L[v // rtiles]) // 64)

@@ -138,7 +138,7 @@ def test_noalloc_rejects_shapes_beyond_its_scratch_before_enqueuing(lib):
     kv = torch.zeros((1, 64, 576), dtype=torch.bfloat16, device=dev)
     bt = torch.zeros((1, 1), dtype=torch.int32, device=dev)
     L = torch.zeros(1, dtype=torch.int32, device=dev)
-    sched = torch.zeros(mla.mla_metadata_size(1, 74) // 4, dtype=torch.int32, device=dev)
+    sched = torch.zeros(mla.mla_metadata_size(1, 1, 128, 74) // 4, dtype=torch.int32, device=dev)
     ns = torch.zeros(2, dtype=torch.int32, device=dev)
     out = torch.zeros((1, 1, 128, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.zeros((1, 1, 128), dtype=torch.float32, device=dev)
