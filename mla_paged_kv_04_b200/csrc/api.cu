@@ -214,6 +214,8 @@ mla_status_t launch_decode_call(const void* q, const void* kv_cache, mla_kv_form
   p.causal = causal ? 1 : 0;
   p.num_parts = num_sm_parts;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.q_wide = aligned(q, 32) ? 1 : 0;
+  p.out_wide = (aligned(out, 32) && aligned(p.o_part, 32)) ? 1 : 0;
   p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   p.trace = g_trace.load(std::memory_order_relaxed);
   {

@@ -99,6 +99,8 @@ struct DecodeParams {
   unsigned long long* trace;    // per-tile timestamps (trace build only), else null
   const int* hold_flag;         // diagnostics (mla_debug_hold_at_tile): device flag, or null
   int hold_tile;                // the PV issuer's tile at which it waits for *hold_flag != 0
+  int q_wide;                   // q is 32-byte aligned: 32-byte loads
+  int out_wide;                 // out and the partials are 32-byte aligned: 32-byte stores
 };
 
 // Per-tile timestamps of the decode kernel, recorded only by a library built
@@ -118,7 +120,8 @@ enum : int {
                        // credit, 5 sent, 6 first half in, 7 P formed, 8 reference
                        // chain, 9 P buffer free, 10 O rescaled, 11 P stored
   kTraceDequant = 4,   // 0 wait for raw bytes, 1 raw ready, 2 stage free, 3 done
-  kTraceItem = 5,      // tile = item: 0 start, 1 Q stored, 2 epilogue start, 3 done
+  kTraceItem = 5,      // tile = item: 0 start, 1 Q stored, 2 epilogue start, 3 done,
+                       // 4 final reference known, 5 row sums joined, 6 last PV done
   kTraceCta = 6,       // tile 0: 0 entry, 1 set up, 2 schedule readable, 3 roles
                        // done, 4 exit, 15 global timer at entry
 };

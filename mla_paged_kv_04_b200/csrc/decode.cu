@@ -65,16 +65,27 @@ constexpr int kRawLatBytes = kPage * 256;               // FP8: this CTA's 256 l
 constexpr int kRawScaleBytes = kPage * 16;              // FP8: the 4 fp32 scales per token
 constexpr int kRawRopeBytes = kPage * 64;               // FP8: this CTA's 32 RoPE bf16 per token
 constexpr int kRawBytes = kRawLatBytes + kRawScaleBytes + kRawRopeBytes;  // 21504
-constexpr int kRawStages = 3;
+#ifndef MLA_FP8_RAW_STAGES
+#define MLA_FP8_RAW_STAGES 2
+#endif
+#ifndef MLA_FP8_STAGES
+#define MLA_FP8_STAGES 3
+#endif
+#ifndef MLA_BF16_STAGES
+#define MLA_BF16_STAGES 5
+#endif
+#ifndef MLA_FP8_XBUFFERS
+#define MLA_FP8_XBUFFERS 3
+#endif
+#ifndef MLA_BF16_XBUFFERS
+#define MLA_BF16_XBUFFERS 2
+#endif
+constexpr int kRawStages = MLA_FP8_RAW_STAGES;
 // Exchange message per tile: fp16 factors [8 chunks of 8 tokens][128 rows][16 B]
 // + the fp32 reference of every row.
 constexpr int kXERegionBytes = 8 * kRows * 16;          // 16384
 constexpr int kXMsgBytes = kXERegionBytes + kRows * 4;  // 16896
 constexpr int kXBufBytes = kXMsgBytes;
-// Two receive buffers, one per softmax warpgroup (tile g uses buffer g % 2).
-// The peer writes tile g + 2's message into buffer g % 2 only after this CTA
-// has read tile g's (a remote arrive on the peer's "buffer free" barrier).
-constexpr int kXBuffers = 2;
 constexpr int kSoftmaxWarps = 8;
 // FP8: one dequant warp per scheduler partition (a warpgroup).
 constexpr int kDqWarps = 4;
@@ -94,7 +105,11 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: the lazy reference mov
 
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kStages = kFp8 ? 3 : 5;  // bf16 page-half stages
+  static constexpr int kStages = kFp8 ? MLA_FP8_STAGES : MLA_BF16_STAGES;  // bf16 page-half stages
+  // Pair-exchange receive buffers: tile g uses buffer g % kXBuffers, and the
+  // peer writes tile g + kXBuffers's message into it only after this CTA has
+  // read tile g's (a remote arrive on the peer's "buffer free" barrier).
+  static constexpr int kXBuffers = kFp8 ? MLA_FP8_XBUFFERS : MLA_BF16_XBUFFERS;
   static constexpr int kThreads = kFp8 ? 384 + 32 * kDqWarps : 384;
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kFull + kStages;
@@ -258,10 +273,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
     mbar_init(BAR(C::kSFree), 4);
     mbar_init(BAR(C::kQReady), kSoftmaxWarps);
-    for (int i = 0; i < 2 * kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
+    for (int i = 0; i < 2 * C::kXBuffers; ++i) mbar_init(BAR(C::kXFull + i), 1);
     mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
     mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
-    for (int i = 0; i < kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
+    for (int i = 0; i < C::kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
     for (int i = 0; i < kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), kDqWarps);
@@ -305,17 +320,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   // workspace and outputs may still be read by the previous combine pass.
   pdl_wait();
   if (threadIdx.x == 0) TRACE(kTraceCta, 0, 2);
-  const int num_parts = p.sched[0];
-  const int32_t* items = p.sched + sched_items_offset(num_parts);
+  // The header and this part's item range are read together (independent
+  // loads, all inside the header of a buffer sized for p.num_parts); the range
+  // is used only if the header matches this call.
+  const int s_parts = p.sched[0], s_vbatch = p.sched[3], s_rtiles = p.sched[7];
+  const int s_first = p.sched[kSchedHeader + part], s_end = p.sched[kSchedHeader + part + 1];
+  const int32_t* items = p.sched + sched_items_offset(p.num_parts);
   int it_begin = 0, it_end = 0;
-  if (num_parts != p.num_parts || p.sched[3] != p.batch * p.row_tiles || p.sched[7] != p.row_tiles) {
+  if (s_parts != p.num_parts || s_vbatch != p.batch * p.row_tiles || s_rtiles != p.row_tiles) {
     // schedule made for another CTA-pair count or another batch: its request
     // ids and item slots may lie outside this call's tensors and workspace,
     // so do nothing and report it
     if (threadIdx.x == 0) report_status(p.status, kStatusBadSchedule);
   } else {
-    it_begin = p.sched[kSchedHeader + part];
-    it_end = p.sched[kSchedHeader + part + 1];
+    it_begin = s_first;
+    it_end = s_end;
   }
 
   // Register budget per warpgroup (FP8, constants above).  The only increase
@@ -339,6 +358,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const int vb = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
         const int b = vb / p.row_tiles, row0 = (vb - b * p.row_tiles) * kRows;
         const int32_t* bt = p.block_table + static_cast<size_t>(b) * p.max_pages;
+        // The block-table entries of the first nst pages, read together and
+        // first of all: at a kernel's start every SM's memory pipe is busy and
+        // a lone dependent load waits for microseconds.  Later entries are
+        // read one page ahead (the wait for a free stage hides the load).
+        // A page past the table's row reads as -1, a bad index.
+        int32_t head[nst];
+#pragma unroll
+        for (int i = 0; i < nst; ++i) head[i] = (p0 + i < p1 && p0 + i < p.max_pages) ? bt[p0 + i] : -1;
+        int32_t bt_next = -1;
         // This producer runs kStages pages ahead: start this item's Q rows
         // towards L2 now, so that the softmax warps' Q loads at the item
         // boundary do not wait on DRAM behind the page stream (rank 0 fetches
@@ -360,7 +388,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           }
           // A page past the block table's row (cache_seqlens larger than
           // 64 * max_pages) is treated like a bad block index.
-          long long phys = pg < p.max_pages ? bt[pg] : -1;
+          const int j = pg - p0;
+          long long phys = bt_next;
+#pragma unroll
+          for (int i = 0; i < nst; ++i)
+            if (j == i) phys = head[i];
+          if (j + 1 >= nst && pg + 1 < p1) bt_next = (pg + 1 < p.max_pages) ? bt[pg + 1] : -1;
           if (phys < 0 || phys >= p.num_blocks) {
             report_status(p.status, kStatusBadBlock);
             phys = 0;
@@ -513,18 +546,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       // go to shared memory (SW64 K-major rows of 64 bytes), warpgroup 1.
       {
         const uint4* qrow = reinterpret_cast<const uint4*>(p.q + orow * kDqk);
-        // all sixteen 16-byte loads first, so their latencies overlap
+        // all loads first, so their latencies overlap: 32-byte loads when q
+        // is 32-byte aligned (rows are 1152 bytes, so then every row is),
+        // else 16-byte ones
         uint32_t v[4][16];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int e0 = static_cast<int>(rank) * 256 + (wg * 4 + c) * 32;
+          if (p.q_wide) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 w = row_ok ? __ldg(qrow + e0 / 8 + u) : make_uint4(0, 0, 0, 0);
-            v[c][4 * u + 0] = w.x;
-            v[c][4 * u + 1] = w.y;
-            v[c][4 * u + 2] = w.z;
-            v[c][4 * u + 3] = w.w;
+            for (int u = 0; u < 2; ++u) {
+              if (row_ok) ld_global_v8(qrow + e0 / 8 + 2 * u, &v[c][8 * u]);
+              else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[c][8 * u + i] = 0u;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 w = row_ok ? __ldg(qrow + e0 / 8 + u) : make_uint4(0, 0, 0, 0);
+              v[c][4 * u + 0] = w.x;
+              v[c][4 * u + 1] = w.y;
+              v[c][4 * u + 2] = w.z;
+              v[c][4 * u + 3] = w.w;
+            }
           }
         }
 #pragma unroll
@@ -604,7 +650,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         ref_own = ref;
         ref_slot[wg * kRows + r] = ref;
         const float msub = (ref == -CUDART_INF_F) ? 0.f : ref;
-        const uint32_t xb = gg & (kXBuffers - 1);
+        constexpr uint32_t kXBuffers = C::kXBuffers;
+        const uint32_t xb = gg % kXBuffers;
         if (wt == 0) {
           mbar_arrive_expect_tx(BAR(C::kXFull + 2 * xb), kXERegionBytes / 2);
           mbar_arrive_expect_tx(BAR(C::kXFull + 2 * xb + 1), kXMsgBytes - kXERegionBytes / 2);
@@ -677,18 +724,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (!ok) break;
         if (wt == 0) TRACE(kTraceSoftmax, gg, 7);
         const float m_new = ref + *reinterpret_cast<const float*>(xs + kXERegionBytes + r * 4);
+        const float rowsum = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
+        {
+          // This warp is done with the peer's message: hand the buffer back
+          // now, before the reference chain.  m_new and rowsum depend on every
+          // value loaded from the buffer, and the arrive's address depends on
+          // both through an opaque zero, so it issues only after those loads
+          // have completed; a relaxed arrive is then enough to keep the peer's
+          // next write behind them.
+          uint32_t z;
+          asm volatile("{\n .reg .b32 t;\n xor.b32 t, %1, %2;\n and.b32 %0, t, 0;\n}\n"
+                       : "=r"(z) : "r"(__float_as_uint(m_new)), "r"(__float_as_uint(rowsum)));
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * xb + z);
+        }
         if (gg > 0 && !warp_wait(BAR(C::kCChain), (gg - 1u) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         if (wt == 0) TRACE(kTraceSoftmax, gg, 8);
         const float m_prev = j > 0 ? comb_slot[r] : -CUDART_INF_F;
         comb_slot[r] = m_new;
         mbar_arrive(BAR(C::kCChain));
-        const float rowsum = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
-        // This warp is done with the peer's message: hand the buffer back.
-        // Every value loaded from it has been consumed by the arithmetic
-        // above (in-order issue), so the loads are complete and a relaxed
-        // arrive is enough to keep the peer's next write behind them.
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * xb);
         const uint32_t pb = gg & 1u;
         // P buffer pb was last read by PV(gg - 2)
         if (gg >= 2) {
@@ -756,17 +810,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (!warp_wait(BAR(C::kCChain), glast & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         m_fin = comb_slot[r];
       }
+      if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 4);
       const float lw = (m_l == -CUDART_INF_F) ? 0.f : l * ex2_approx(m_l - m_fin);
       epi_slot[wg * kRows + r] = lw;
       ref_slot[wg * kRows + r] = -CUDART_INF_F;  // the next item starts afresh
       mbar_arrive(BAR(C::kEpi));
       if (!warp_wait(BAR(C::kEpi), nitem & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+      if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 5);
       ++nitem;
       const float lt = lw + epi_slot[(wg ^ 1) * kRows + r];
       if (!warp_wait(BAR(C::kPvDone + (glast & 1u)), (glast >> 1) & 1u, abort_flag, p.timeout_ns)) {
         ok = false;
         break;
       }
+      if (wg == 0 && wt == 0) TRACE(kTraceItem, it - it_begin, 6);
       tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const float lse_val = lt > 0.f ? (m_fin + __log2f(lt)) * 0.69314718055994531f : -CUDART_INF_F;
@@ -776,22 +833,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const int col = wg * 128 + cc * 32;  // within this CTA's 256 columns
         tmem_ld32(trow + kColO + col, o);
         if (row_ok) {
+          // Each thread writes its own row: 32-byte stores (a whole sector
+          // per lane) when the buffers allow, else 16-byte ones.
           if (slot < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + orow * kDv + rank * 256 + col);
+            uint16_t* dst = p.out + orow * kDv + rank * 256 + col;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              dst[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
-                                  pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
-                                  pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
-                                  pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+            for (int h = 0; h < 2; ++h) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack_bf16x2(__uint_as_float(o[16 * h + 2 * i]) * inv, __uint_as_float(o[16 * h + 2 * i + 1]) * inv);
+              if (p.out_wide) {
+                st_global_v8(dst + 16 * h, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+              } else {
+                uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * h);
+                d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              }
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(slot) * mt + r) * kDv +
-                                                    rank * 256 + col);
+            float* dst = p.o_part + (static_cast<size_t>(slot) * mt + r) * kDv + rank * 256 + col;
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                   __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv);
+            if (p.out_wide) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                st_global_v8(dst + 8 * v, o[8 * v], o[8 * v + 1], o[8 * v + 2], o[8 * v + 3], o[8 * v + 4],
+                             o[8 * v + 5], o[8 * v + 6], o[8 * v + 7]);
+            } else {
+              float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                d4[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                    __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+            }
           }
         }
       }

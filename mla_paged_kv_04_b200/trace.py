@@ -121,12 +121,16 @@ def summarize(ts: np.ndarray, skip: int = 4) -> dict:
     for c in range(ts.shape[0]):
         for it in range(TILES):
             e = ts[c, ITEM, it].astype(np.int64)
-            if e[0] > 0 and e[3] > 0:
-                items.append((e[1] - e[0], e[3] - e[2]))
+            if e[0] > 0 and e[3] > 0 and e[6] > 0:
+                items.append((e[1] - e[0], e[3] - e[2], e[4] - e[2], e[5] - e[4], e[6] - e[5], e[3] - e[6]))
     if items:
         s = np.median(np.array(items, dtype=np.float64), axis=0)
         out["item: Q load"] = float(s[0])
         out["item: epilogue"] = float(s[1])
+        out["item: epilogue, final reference"] = float(s[2])
+        out["item: epilogue, row sums joined"] = float(s[3])
+        out["item: epilogue, last PV done"] = float(s[4])
+        out["item: epilogue, O out"] = float(s[5])
     return out
 
 
