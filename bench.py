@@ -14,7 +14,8 @@ Prints ONE JSON line on rank 0.  By default the line's top-level numbers are
 those of the FP8 656-byte-cache workload (b=128, h_q=128, L ~ U[16384, 32768],
 the compute-bound configuration) in TFLOP/s, and `per_config` holds the same
 record for the four other workloads.  For each workload:
-  value        algorithmic flops / (time of the K timed steps / K)
+  value        algorithmic flops / (time of the K timed steps / K); a step
+               replays a CUDA graph of schedule + decode + combine
   roofline     the decode call alone (decode + combine kernels), median of at
                least 50 calls each after an L2 flush, against the measured
                peak of the bound (tensor or HBM)
@@ -80,6 +81,24 @@ def algorithmic_work(w: W.Workload, seqlens: np.ndarray):
         vis += int(np.clip(L - w.s_q + i + 1, 0, None).sum()) if w.causal else int(L.sum())
     flops = 2 * (576 + 512) * w.h_q * vis
     return dict(bytes=kv + q + out + lse + meta, kv_bytes=kv, flops=flops)
+
+
+def sparse_work(w: W.Workload, seqlens: np.ndarray, indices: np.ndarray):
+    """Bytes and flops of one sparse decode: every valid list entry (0 <= idx < L)
+    is one key read (656 bytes) and one (query token, key) pair per head.
+
+    bytes = 656 * valid + |q| + |out| + |lse| + 4 * |indices| + 4 * valid
+            (block-table entries) + 4 b (lengths)
+    flops = 2 * (576 + 512) * h_q * valid
+    """
+    L = seqlens.astype(np.int64)[:, None, None]
+    valid = int(((indices >= 0) & (indices < L)).sum())
+    B = L.shape[0]
+    q = B * w.s_q * w.h_q * 576 * 2
+    out = B * w.s_q * w.h_q * 512 * 2
+    lse = B * w.s_q * w.h_q * 4
+    nbytes = 656 * valid + q + out + lse + 4 * indices.size + 4 * valid + 4 * B
+    return dict(bytes=nbytes, kv_bytes=656 * valid, flops=2 * (576 + 512) * w.h_q * valid)
 
 
 def kernel_source_hash() -> str:
@@ -200,14 +219,23 @@ def oracle_rate(w: W.Workload, budget_s: float = 12.0, seed: int = 0):
     import oracle
     pool = []
     for b in range(4):
-        one = W.Workload(w.name, 1, w.s_q, w.h_q, w.seqlen, fmt=w.fmt, causal=w.causal, seed=seed + b)
-        a = W.oracle_arrays(W.make_case(one, poison=False))
-        work = algorithmic_work(one, a["cache_seqlens"])
+        one = W.Workload(w.name, 1, w.s_q, w.h_q, w.seqlen, fmt=w.fmt, causal=w.causal, seed=seed + b, topk=w.topk)
+        case = W.make_case(one, poison=False)
+        a = W.oracle_arrays(case)
+        if w.topk:
+            a["indices"] = case["indices"].numpy()
+            work = sparse_work(one, a["cache_seqlens"], a["indices"])
+        else:
+            work = algorithmic_work(one, a["cache_seqlens"])
         pool.append((a, work["bytes"], work["flops"]))
 
     def call(a):
-        oracle.mla_decode(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
-                          a["softmax_scale"], a["causal"])
+        if w.topk:
+            oracle.mla_sparse_decode(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
+                                     a["indices"], a["softmax_scale"])
+        else:
+            oracle.mla_decode(a["q_bits"], a["kv_cache"], a["fmt"], a["block_table"], a["cache_seqlens"],
+                              a["softmax_scale"], a["causal"])
 
     call(pool[0][0])
     n_done, t_total, bytes_done, flops_done = 0, 0.0, 0, 0
@@ -301,7 +329,7 @@ def run_reference(args, world, rank):
 
 
 HEADLINE = "fp8_656"          # the compute-bound configuration (FP8 656-byte cache)
-PER_CONFIG = ["tiny", "uniform_bf16", "varlen_spec_bf16", "long_ctx_bf16"]
+PER_CONFIG = ["tiny", "uniform_bf16", "varlen_spec_bf16", "long_ctx_bf16", "sparse_fp8"]
 MIN_REPS = 50                 # decode calls timed for the roofline, at least (a short burst: a
                               # loop of seconds runs into the power cap and measures that instead)
 
@@ -324,15 +352,31 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
     lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     seqlens_np = L.cpu().numpy()
-    work = algorithmic_work(w, seqlens_np)
     stream = torch.cuda.current_stream(dev)
+    if w.topk:
+        # the sparse decode over the same kind of cache: its own schedule and workspace
+        idx = case["indices"]
+        work = sparse_work(w, seqlens_np, idx.cpu().numpy())
+        sched = torch.empty(mla.mla_sparse_metadata_size_bytes(B, s_q, h_q, parts) // 4, dtype=torch.int32,
+                            device=dev)
+        ns = torch.empty(mla.mla_sparse_num_splits_len(B, s_q, h_q), dtype=torch.int32, device=dev)
+        ws = torch.zeros(mla.mla_sparse_workspace_size(B, s_q, h_q, parts), dtype=torch.uint8, device=dev)
 
-    def meta():
-        mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
+        def meta(st=stream):
+            mla.mla_get_sparse_metadata(B, s_q, h_q, w.topk, parts, device=dev, sched=sched, num_splits=ns,
+                                        stream=st)
 
-    def decode():
-        mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
-                           stream=stream)
+        def decode(st=stream):
+            mla.mla_sparse_decode_fwd(q, kv, bt, L, idx, w.softmax_scale, sched, ns, parts, out, lse, ws, stream=st)
+    else:
+        work = algorithmic_work(w, seqlens_np)
+
+        def meta(st=stream):
+            mla.mla_get_metadata(L, s_q, h_q, parts, sched=sched, num_splits=ns, stream=st)
+
+        def decode(st=stream):
+            mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws,
+                               stream=st)
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
@@ -344,6 +388,36 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
         raise SystemExit(f"{w.name}: device status {mla.STATUS.get(status, status)} during warm-up")
 
     reps = max(MIN_REPS, args.steps)
+
+    # The calls are replayed from CUDA graphs, captured once through the
+    # public API: a step's kernels then reach the GPU back to back, and the
+    # event pair measures the GPU's time, not the host's launch overhead
+    # (for small batches the host is slower than the kernels).  The L2 flush
+    # runs before each timed step, outside the graph and the event pair.
+    #   g_step: schedule + decode + combine (one step of the hot path)
+    #   g_call: decode + combine (the decode call, for the roofline)
+    #   g_meta: the schedule alone
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    g_step, g_call, g_meta = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    meta_c = lambda: meta(cap)
+    decode_c = lambda: decode(cap)
+    with torch.cuda.stream(cap):
+        meta_c()
+        decode_c()
+    cap.synchronize()
+    with torch.cuda.graph(g_step, stream=cap):
+        meta_c()
+        decode_c()
+    with torch.cuda.graph(g_call, stream=cap):
+        decode_c()
+    with torch.cuda.graph(g_meta, stream=cap):
+        meta_c()
+    stream.wait_stream(cap)
+    for _ in range(3):
+        flush.zero_()
+        g_step.replay()
+    torch.cuda.synchronize(dev)
 
     # The timed steps: one event pair per step around the whole hot path
     # (schedule + decode + combine), L2 flushed before each.  No event sits
@@ -358,16 +432,15 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
-            meta()
-            decode()
+            g_step.replay()
             ev[i][1].record(stream)
         # The decode call alone (decode + combine kernels), for the roofline:
         # the median of `reps` calls, each after an L2 flush and the schedule.
         for i in range(reps):
             flush.zero_()
-            meta()
+            g_meta.replay()
             dec_ev[i][0].record(stream)
-            decode()
+            g_call.replay()
             dec_ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
@@ -377,10 +450,11 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
     for i in range(MIN_REPS):  # the schedule kernel alone
         flush.zero_()
         meta_ev[i][0].record(stream)
-        meta()
+        g_meta.replay()
         meta_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     meta_ms = [e[0].elapsed_time(e[1]) for e in meta_ev]
+    del g_step, g_call, g_meta
     status = mla.mla_last_device_status(ws)
     if status != 0:
         raise SystemExit(f"{w.name}: device status {mla.STATUS.get(status, status)} in the timed region")
@@ -404,6 +478,10 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
     out_d = [out, torch.empty_like(out)]
     lse_d = [lse, torch.empty_like(lse)]
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + L_h.numel() * 4
+    if w.topk:
+        idx_h = idx.cpu().pin_memory()
+        idx_d = [torch.empty_like(idx) for _ in range(2)]
+        h2d += idx_h.numel() * 4
     d2h = out_h[0].numel() * 2 + lse_h[0].numel() * 4
     s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     up_done = [torch.cuda.Event() for _ in range(2)]
@@ -417,13 +495,21 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
             q_d[k].copy_(q_h, non_blocking=True)
             bt_d[k].copy_(bt_h, non_blocking=True)
             L_d[k].copy_(L_h, non_blocking=True)
+            if w.topk:
+                idx_d[k].copy_(idx_h, non_blocking=True)
             up_done[k].record(s_up)
         stream.wait_event(up_done[k])
         stream.wait_event(dn_done[k])  # step i - 2's results have left buffer k
         flush.zero_()
-        mla.mla_get_metadata(L_d[k], s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
-        mla.mla_decode_fwd(q_d[k], kv, w.fmt, bt_d[k], L_d[k], w.softmax_scale, w.causal, sched, ns, parts,
-                           out_d[k], lse_d[k], ws, stream=stream)
+        if w.topk:
+            mla.mla_get_sparse_metadata(B, s_q, h_q, w.topk, parts, device=dev, sched=sched, num_splits=ns,
+                                        stream=stream)
+            mla.mla_sparse_decode_fwd(q_d[k], kv, bt_d[k], L_d[k], idx_d[k], w.softmax_scale, sched, ns, parts,
+                                      out_d[k], lse_d[k], ws, stream=stream)
+        else:
+            mla.mla_get_metadata(L_d[k], s_q, h_q, parts, sched=sched, num_splits=ns, stream=stream)
+            mla.mla_decode_fwd(q_d[k], kv, w.fmt, bt_d[k], L_d[k], w.softmax_scale, w.causal, sched, ns, parts,
+                               out_d[k], lse_d[k], ws, stream=stream)
         cmp_done[k].record(stream)
         with torch.cuda.stream(s_dn):
             s_dn.wait_event(cmp_done[k])
@@ -519,6 +605,7 @@ def run_cuda(args, world, rank, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(rec["config"], **{
             "mma": "bf16 operands (FP8 cache dequantised in shared memory), fp32 accumulation",
+            "launch": "each timed step replays a CUDA graph of the public calls (schedule, decode, combine)",
             "l2": "flushed before every timed step and every roofline rep (256 MiB write)",
             "parallelism": f"replicas x{n} (independent request batches)"}),
         "gbs": rec["gbs"],
@@ -549,15 +636,22 @@ def run_trace(args):
     q, kv, bt, L = case["q"], case["kv_cache"], case["block_table"], case["cache_seqlens"]
     B = case["batch"]
     parts = args.parts or mla.mla_default_num_sm_parts(dev)
-    sched, ns = mla.mla_get_metadata(L, w.s_q, w.h_q, parts)
-    ws = mla.alloc_workspace(B, w.s_q, w.h_q, parts, dev)
     out = torch.empty((B, w.s_q, w.h_q, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, w.s_q, w.h_q), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if w.topk:
+        sched, ns = mla.mla_get_sparse_metadata(B, w.s_q, w.h_q, w.topk, parts, device=dev)
+        ws = torch.zeros(mla.mla_sparse_workspace_size(B, w.s_q, w.h_q, parts), dtype=torch.uint8, device=dev)
+    else:
+        sched, ns = mla.mla_get_metadata(L, w.s_q, w.h_q, parts)
+        ws = mla.alloc_workspace(B, w.s_q, w.h_q, parts, dev)
 
     def run():
         flush.zero_()
-        mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws)
+        if w.topk:
+            mla.mla_sparse_decode_fwd(q, kv, bt, L, case["indices"], w.softmax_scale, sched, ns, parts, out, lse, ws)
+        else:
+            mla.mla_decode_fwd(q, kv, w.fmt, bt, L, w.softmax_scale, w.causal, sched, ns, parts, out, lse, ws)
 
     for _ in range(3):
         run()

@@ -155,6 +155,51 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sparse decode over the 656-byte FP8 cache.  The menfem.com DeepSeek page
+ * ("Key Contributions") names a sparse decode kernel over this cache format
+ * (250 -> 410 TFLOPS on H800, up to 350 TFLOPS on B200) without defining
+ * it; this library's reading:
+ *
+ *   For request b, query token i in [0, s_q) and head h, with
+ *   L = cache_seqlens[b] and the list idx = indices[b, i, 0:topk]:
+ *     the keys are K_{idx_k} for every entry with 0 <= idx_k < L (the same
+ *     positions the dense decode reads through block_table); entries outside
+ *     [0, L) are padding and are not keys; an entry listed twice is two
+ *     terms.  There is no causal mask: the list decides what is visible.
+ *     x_k = softmax_scale * q[b,i,h,:] . K_{idx_k}
+ *     lse[b,i,h] = ln sum_k exp(x_k),  out[b,i,h,:] = sum_k exp(x_k - lse) V_{idx_k}
+ *   A row with no valid entry gets out = 0 and lse = -inf.
+ *
+ *   q              device bf16 [batch, s_q, h_q, 576]; h_q <= 1024
+ *   kv_cache       device uint8 [num_blocks, 64, 656], 16-byte aligned
+ *   block_table    device int32 [batch, max_pages]
+ *   cache_seqlens  device int32 [batch]
+ *   indices        device int32 [batch, s_q, topk], 4-byte aligned
+ *   topk           entries per list, 1 <= topk <= 2^24
+ *   sched, num_splits  from mla_get_sparse_metadata (same batch, s_q, h_q,
+ *                  topk, num_sm_parts): a schedule of batch * s_q units of
+ *                  h_q rows, each of length topk
+ *   out, lse       as mla_decode_fwd;  workspace >= mla_sparse_workspace_size()
+ * Each CTA pair gathers the listed tokens of a 64-entry tile with bulk
+ * copies (this CTA's 336 bytes of each token), dequantises them like the
+ * dense FP8 decode and runs the same MMA and softmax pipeline.  Device-
+ * detected errors as mla_decode_fwd (a listed position whose page maps
+ * outside [0, num_blocks): MLA_ERR_BAD_BLOCK_INDEX, that entry left out).
+ */
+int mla_sparse_num_splits_len(int batch, int s_q, int h_q);
+size_t mla_sparse_metadata_size(int batch, int s_q, int h_q, int num_sm_parts);
+size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int num_sm_parts);
+mla_status_t mla_get_sparse_metadata(int batch, int s_q, int h_q, int topk, int num_sm_parts,
+                                     int32_t* sched, int32_t* num_splits, void* stream);
+mla_status_t mla_sparse_decode_fwd(const void* q, const void* kv_cache, int64_t num_blocks,
+                                   const int32_t* block_table, int max_pages,
+                                   const int32_t* cache_seqlens, const int32_t* indices, int topk,
+                                   int batch, int s_q, int h_q, float softmax_scale,
+                                   const int32_t* sched, const int32_t* num_splits, int num_sm_parts,
+                                   void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
  * Cache append: write new tokens into the paged cache, the step that fills
  * what mla_decode_fwd reads.  The pages print only the FP8 token's size (656
  * bytes against 1,152 in BF16, RoPE slice kept in BF16: menfem.com DeepSeek

@@ -10,9 +10,10 @@ Names follow the C ABI:
   mla_workspace_size, mla_decode_fwd, mla_decode_fwd_noalloc,
   mla_noalloc_last_device_status, mla_kv_append, mla_last_device_status,
   mla_clear_device_status, mla_status_string, mla_set_wait_timeout_ns,
-  mla_debug_trace_bytes, mla_debug_set_trace_buffer, mla_debug_hold_at_tile
-plus `decode(...)`, a convenience wrapper that allocates the outputs, the
-schedule and the workspace.  Every tensor argument is checked (device, dtype,
+  mla_debug_trace_bytes, mla_debug_set_trace_buffer, mla_debug_hold_at_tile,
+  mla_get_sparse_metadata, mla_sparse_workspace_size, mla_sparse_decode_fwd
+plus `decode(...)` and `sparse_decode(...)`, convenience wrappers that
+allocate the outputs, the schedule and the workspace.  Every tensor argument is checked (device, dtype,
 shape, size) before its pointer reaches the C ABI.
 """
 
@@ -75,6 +76,17 @@ def load_library(trace: bool = False):
     lib.mla_decode_fwd_noalloc.restype = c_int
     lib.mla_decode_fwd_noalloc.argtypes = [vp, vp, c_int, c_i64, vp, c_int, vp, c_int, c_int, c_int, c_float, c_int,
                                            vp, vp, c_int, vp, vp, vp]
+    lib.mla_sparse_num_splits_len.restype = c_int
+    lib.mla_sparse_num_splits_len.argtypes = [c_int, c_int, c_int]
+    lib.mla_sparse_metadata_size.restype = c_size
+    lib.mla_sparse_metadata_size.argtypes = [c_int, c_int, c_int, c_int]
+    lib.mla_sparse_workspace_size.restype = c_size
+    lib.mla_sparse_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+    lib.mla_get_sparse_metadata.restype = c_int
+    lib.mla_get_sparse_metadata.argtypes = [c_int, c_int, c_int, c_int, c_int, vp, vp, vp]
+    lib.mla_sparse_decode_fwd.restype = c_int
+    lib.mla_sparse_decode_fwd.argtypes = [vp, vp, c_i64, vp, c_int, vp, vp, c_int, c_int, c_int, c_int, c_float,
+                                          vp, vp, c_int, vp, vp, vp, c_size, vp]
     lib.mla_kv_append.restype = c_int
     lib.mla_kv_append.argtypes = [vp, c_int, c_int, vp, vp, c_int, vp, c_int, c_i64, vp, c_size, vp]
     lib.mla_last_device_status.restype = c_int
@@ -122,6 +134,8 @@ def _on_device(device: torch.device, **tensors):
     the C ABI receives bare pointers and cannot tell."""
     if device.type != "cuda":
         raise ValueError(f"tensors must be CUDA tensors, got {device}")
+    if device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
     for name, t in tensors.items():
         if not isinstance(t, torch.Tensor):
             raise TypeError(f"{name} must be a torch.Tensor")
@@ -266,6 +280,97 @@ def mla_decode_fwd_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, fmt: str, bl
                                       h_q, float(softmax_scale), 1 if causal else 0, sched.data_ptr(),
                                       num_splits.data_ptr(), int(num_sm_parts), out.data_ptr(), lse.data_ptr(),
                                       _stream(stream)), "mla_decode_fwd_noalloc")
+    return out, lse
+
+
+def mla_get_sparse_metadata(batch: int, s_q: int, h_q: int, topk: int, num_sm_parts: int | None = None,
+                            device=None, sched: torch.Tensor | None = None, num_splits: torch.Tensor | None = None,
+                            stream=None):
+    """Split-KV schedule of a sparse decode: batch * s_q units of h_q rows,
+    each attending to topk list entries -> (sched, num_splits)."""
+    lib = _active_lib()
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    parts = mla_default_num_sm_parts(device) if num_sm_parts is None else int(num_sm_parts)
+    nbytes = lib.mla_sparse_metadata_size(batch, s_q, h_q, parts)
+    n_len = lib.mla_sparse_num_splits_len(batch, s_q, h_q)
+    if nbytes == 0 or n_len == 0:
+        raise MLAError(2, "mla_get_sparse_metadata")
+    if sched is None:
+        sched = torch.empty(max(nbytes // 4, 1), dtype=torch.int32, device=device)
+    if num_splits is None:
+        num_splits = torch.empty(n_len, dtype=torch.int32, device=device)
+    _on_device(device, sched=sched, num_splits=num_splits)
+    if sched.dtype != torch.int32 or num_splits.dtype != torch.int32 or num_splits.numel() < n_len or \
+            _nbytes(sched) < nbytes:
+        raise ValueError(f"sched (int32, >= {nbytes} bytes) and num_splits (int32, >= {n_len}) too small")
+    _check(lib.mla_get_sparse_metadata(batch, s_q, h_q, int(topk), parts, sched.data_ptr(), num_splits.data_ptr(),
+                                       _stream(stream)), "mla_get_sparse_metadata")
+    return sched, num_splits
+
+
+def mla_sparse_workspace_size(batch: int, s_q: int, h_q: int, num_sm_parts: int) -> int:
+    return _active_lib().mla_sparse_workspace_size(batch, s_q, h_q, num_sm_parts)
+
+
+def mla_sparse_metadata_size_bytes(batch: int, s_q: int, h_q: int, num_sm_parts: int) -> int:
+    return _active_lib().mla_sparse_metadata_size(batch, s_q, h_q, num_sm_parts)
+
+
+def mla_sparse_num_splits_len(batch: int, s_q: int, h_q: int) -> int:
+    return _active_lib().mla_sparse_num_splits_len(batch, s_q, h_q)
+
+
+def mla_sparse_decode_fwd(q: torch.Tensor, kv_cache: torch.Tensor, block_table: torch.Tensor,
+                          cache_seqlens: torch.Tensor, indices: torch.Tensor, softmax_scale: float,
+                          sched: torch.Tensor, num_splits: torch.Tensor, num_sm_parts: int, out: torch.Tensor,
+                          lse: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """Enqueue the sparse decode (FP8 656-byte cache): query token i of request
+    b attends to the positions indices[b, i, :] (entries outside [0, L) are
+    padding); see include/mla.h."""
+    lib = _active_lib()
+    if q.dim() != 4 or q.shape[3] != 576 or q.dtype != torch.bfloat16:
+        raise ValueError(f"q must be bf16 [batch, s_q, h_q, 576], got {q.dtype} {tuple(q.shape)}")
+    B, s_q, h_q, _ = q.shape
+    _on_device(q.device, q=q, kv_cache=kv_cache, block_table=block_table, cache_seqlens=cache_seqlens,
+               indices=indices, sched=sched, num_splits=num_splits, out=out, lse=lse, workspace=workspace)
+    _check_cache(kv_cache, "fp8_656")
+    if indices.dtype != torch.int32 or indices.dim() != 3 or tuple(indices.shape[:2]) != (B, s_q):
+        raise ValueError(f"indices must be int32 [{B}, {s_q}, topk], got {indices.dtype} {tuple(indices.shape)}")
+    topk = indices.shape[2]
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be int32 [batch={B}, max_pages]")
+    if cache_seqlens.dtype != torch.int32 or cache_seqlens.numel() != B:
+        raise ValueError(f"cache_seqlens must be int32 [{B}]")
+    if out.shape != (B, s_q, h_q, 512) or out.dtype != torch.bfloat16:
+        raise ValueError(f"out must be bf16 {(B, s_q, h_q, 512)}")
+    if lse.shape != (B, s_q, h_q) or lse.dtype != torch.float32:
+        raise ValueError(f"lse must be fp32 {(B, s_q, h_q)}")
+    nbytes = lib.mla_sparse_metadata_size(B, s_q, h_q, int(num_sm_parts))
+    if sched.dtype != torch.int32 or _nbytes(sched) < nbytes or num_splits.dtype != torch.int32 or \
+            num_splits.numel() < lib.mla_sparse_num_splits_len(B, s_q, h_q):
+        raise ValueError("sched / num_splits do not fit this shape (use mla_get_sparse_metadata)")
+    _check(lib.mla_sparse_decode_fwd(q.data_ptr(), kv_cache.data_ptr(), kv_cache.shape[0], block_table.data_ptr(),
+                                     block_table.shape[1], cache_seqlens.data_ptr(), indices.data_ptr(), topk, B,
+                                     s_q, h_q, float(softmax_scale), sched.data_ptr(), num_splits.data_ptr(),
+                                     int(num_sm_parts), out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                     _nbytes(workspace), _stream(stream)), "mla_sparse_decode_fwd")
+    return out, lse
+
+
+def sparse_decode(q, kv_cache, block_table, cache_seqlens, indices, softmax_scale, num_sm_parts=None, stream=None):
+    """One-shot sparse decode: schedule + workspace + outputs allocated here -> (out, lse)."""
+    B, s_q, h_q, _ = q.shape
+    parts = mla_default_num_sm_parts(q.device) if num_sm_parts is None else int(num_sm_parts)
+    sched, num_splits = mla_get_sparse_metadata(B, s_q, h_q, indices.shape[2], parts, device=q.device,
+                                                stream=stream)
+    n = mla_sparse_workspace_size(B, s_q, h_q, parts)
+    if n == 0:
+        raise MLAError(2, "mla_sparse_workspace_size")
+    ws = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    out = torch.empty((B, s_q, h_q, 512), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=q.device)
+    mla_sparse_decode_fwd(q, kv_cache, block_table, cache_seqlens, indices, softmax_scale, sched, num_splits, parts,
+                          out, lse, ws, stream=stream)
     return out, lse
 
 

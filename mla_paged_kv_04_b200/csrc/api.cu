@@ -16,14 +16,16 @@
 #include "entry.cuh"
 
 namespace mla {
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int rtiles, int parts, int32_t* sched,
-                            int32_t* num_splits, cudaStream_t stream);
+cudaError_t launch_metadata(const int32_t* seqlens, int uniform_len, int batch, int rtiles, int parts,
+                            int32_t* sched, int32_t* num_splits, cudaStream_t stream);
 int metadata_max_batch();
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream);
 cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
                                int num_parts, cudaStream_t stream);
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_scale, const CUtensorMap& tm_rope,
                               const DecodeParams& p, int num_parts, cudaStream_t stream);
+cudaError_t launch_decode_sparse_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_tail, const DecodeParams& p,
+                                     int num_parts, cudaStream_t stream);
 }  // namespace mla
 
 using namespace mla;
@@ -31,6 +33,7 @@ using namespace mla;
 namespace {
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr int kMaxTopk = 1 << 24;  // sparse decode: entries per index list
 
 // Limit of every bounded wait in the decode kernel (mla_set_wait_timeout_ns).
 std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
@@ -150,7 +153,7 @@ mla_status_t mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, 
   mla_status_t st = check_shape(batch, s_q, h_q);
   if (st != MLA_OK) return st;
   const int rt = row_tiles(s_q * h_q);
-  cudaError_t e = launch_metadata(cache_seqlens, batch * rt, rt, num_sm_parts, sched, num_splits,
+  cudaError_t e = launch_metadata(cache_seqlens, 0, batch * rt, rt, num_sm_parts, sched, num_splits,
                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -214,6 +217,8 @@ mla_status_t launch_decode_call(const void* q, const void* kv_cache, mla_kv_form
   p.causal = causal ? 1 : 0;
   p.num_parts = num_sm_parts;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.req_div = 1;
+  p.req_batch = batch;
   p.q_wide = aligned(q, 32) ? 1 : 0;
   p.out_wide = (aligned(out, 32) && aligned(p.o_part, 32)) ? 1 : 0;
   p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
@@ -279,6 +284,116 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
   if (!device_supported()) return MLA_ERR_UNSUPPORTED;
   return launch_decode_call(q, kv_cache, fmt, num_blocks, block_table, max_pages, cache_seqlens, batch, s_q, h_q,
                             softmax_scale, causal, sched, num_splits, num_sm_parts, out, lse, workspace, stream);
+}
+
+int mla_sparse_num_splits_len(int batch, int s_q, int h_q) {
+  if (batch < 1 || s_q < 1 || static_cast<long long>(batch) * s_q > (1 << 30)) return 0;
+  return mla_num_splits_len(batch * s_q, 1, h_q);
+}
+
+size_t mla_sparse_metadata_size(int batch, int s_q, int h_q, int num_sm_parts) {
+  if (batch < 1 || s_q < 1 || static_cast<long long>(batch) * s_q > (1 << 30)) return 0;
+  return mla_metadata_size(batch * s_q, 1, h_q, num_sm_parts);
+}
+
+size_t mla_sparse_workspace_size(int batch, int s_q, int h_q, int num_sm_parts) {
+  if (batch < 1 || s_q < 1 || static_cast<long long>(batch) * s_q > (1 << 30)) return 0;
+  return mla_workspace_size(batch * s_q, 1, h_q, num_sm_parts);
+}
+
+mla_status_t mla_get_sparse_metadata(int batch, int s_q, int h_q, int topk, int num_sm_parts, int32_t* sched,
+                                     int32_t* num_splits, void* stream) {
+  if (!sched || !num_splits || !aligned(sched, 16) || !aligned(num_splits, 4)) return MLA_ERR_INVALID_ARG;
+  if (num_sm_parts < 1 || num_sm_parts > 65535 || topk < 1 || topk > kMaxTopk) return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || s_q < 1) return MLA_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * s_q > (1 << 30)) return MLA_ERR_UNSUPPORTED;
+  const int units = batch * s_q;
+  mla_status_t st = check_shape(units, 1, h_q);
+  if (st != MLA_OK) return st;
+  const int rt = row_tiles(h_q);
+  cudaError_t e = launch_metadata(nullptr, topk, units * rt, rt, num_sm_parts, sched, num_splits,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_sparse_decode_fwd(const void* q, const void* kv_cache, int64_t num_blocks,
+                                   const int32_t* block_table, int max_pages, const int32_t* cache_seqlens,
+                                   const int32_t* indices, int topk, int batch, int s_q, int h_q, float softmax_scale,
+                                   const int32_t* sched, const int32_t* num_splits, int num_sm_parts, void* out,
+                                   float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!indices || !aligned(indices, 4) || topk < 1 || topk > kMaxTopk) return MLA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || s_q < 1) return MLA_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * s_q > (1 << 30)) return MLA_ERR_UNSUPPORTED;
+  const int units = batch * s_q;
+  // the unit checks of a dense call with `units` requests of h_q rows
+  mla_status_t st = check_decode_args(q, kv_cache, MLA_KV_FP8_656, num_blocks, block_table, max_pages,
+                                      cache_seqlens, units, 1, h_q, softmax_scale, sched, num_splits, num_sm_parts,
+                                      out, lse);
+  if (st != MLA_OK) return st;
+  if (workspace_bytes < ws_bytes(units, num_sm_parts, h_q)) return MLA_ERR_WORKSPACE;
+  if (!device_supported()) return MLA_ERR_UNSUPPORTED;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.sched = sched;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.lse_part = reinterpret_cast<float*>(ws + ws_lse_offset());
+  p.o_part = reinterpret_cast<float*>(ws + ws_o_offset(units, num_sm_parts, h_q));
+  p.status = reinterpret_cast<int*>(ws);
+  p.num_blocks = num_blocks;
+  p.max_pages = max_pages;
+  p.batch = units;
+  p.s_q = 1;
+  p.h_q = h_q;
+  p.M = h_q;
+  p.row_tiles = row_tiles(h_q);
+  p.causal = 0;
+  p.num_parts = num_sm_parts;
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
+  p.req_div = s_q;
+  p.req_batch = batch;
+  p.kv_raw = static_cast<const uint8_t*>(kv_cache);
+  p.indices = indices;
+  p.topk = topk;
+  p.q_wide = aligned(q, 32) ? 1 : 0;
+  p.out_wide = (aligned(out, 32) && aligned(p.o_part, 32)) ? 1 : 0;
+  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  p.trace = g_trace.load(std::memory_order_relaxed);
+  {
+    std::lock_guard<std::mutex> lock(g_hold_mutex);
+    p.hold_flag = g_hold_flag;
+    p.hold_tile = g_hold_tile;
+  }
+  // one-row boxes for the TMA row gathers: this CTA's latent half (256 bytes)
+  // and bytes [496, 656) of the token
+  const uint64_t rows = static_cast<uint64_t>(num_blocks) * kPage;
+  CUtensorMap tm_lat, tm_tail;
+  if (!make_map(&tm_lat, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 256, 1,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&tm_tail, CU_TENSOR_MAP_DATA_TYPE_UINT8, kv_cache, kFp8TokenBytes, rows, kFp8TokenBytes, 160, 1,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return MLA_ERR_CUDA;
+  cudaError_t e = launch_decode_sparse_fp8(tm_lat, tm_tail, p, num_sm_parts, s);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  CombineParams c{};
+  c.sched = sched;
+  c.num_splits = num_splits;
+  c.lse_part = p.lse_part;
+  c.o_part = p.o_part;
+  c.out = p.out;
+  c.lse = lse;
+  c.batch = units;
+  c.M = h_q;
+  c.row_tiles = p.row_tiles;
+  c.num_parts = num_sm_parts;
+  e = launch_combine(c, num_sm_parts, s);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status_t mla_kv_append(const void* kv_new, int batch, int s_new, const int32_t* cache_seqlens,

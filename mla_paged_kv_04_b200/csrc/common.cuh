@@ -101,6 +101,15 @@ struct DecodeParams {
   int hold_tile;                // the PV issuer's tile at which it waits for *hold_flag != 0
   int q_wide;                   // q is 32-byte aligned: 32-byte loads
   int out_wide;                 // out and the partials are 32-byte aligned: 32-byte stores
+  // Units and requests.  Rows of q, out and lse are grouped in `batch` units
+  // of M rows.  Dense decode: a unit is a request (req_div = 1).  Sparse
+  // decode: a unit is one query token of a request (M = h_q, req_div = s_q),
+  // and the block table and the lengths are indexed by unit / req_div.
+  int req_div;
+  int req_batch;                // rows of block_table and seqlens
+  const uint8_t* kv_raw;        // sparse: the 656-byte cache, read with bulk copies
+  const int32_t* indices;       // sparse: [batch units, topk] positions in the request
+  int topk;
 };
 
 // Per-tile timestamps of the decode kernel, recorded only by a library built

@@ -65,6 +65,14 @@ constexpr int kRawLatBytes = kPage * 256;               // FP8: this CTA's 256 l
 constexpr int kRawScaleBytes = kPage * 16;              // FP8: the 4 fp32 scales per token
 constexpr int kRawRopeBytes = kPage * 64;               // FP8: this CTA's 32 RoPE bf16 per token
 constexpr int kRawBytes = kRawLatBytes + kRawScaleBytes + kRawRopeBytes;  // 21504
+// Sparse decode: the gather brings, per token, this CTA's latent half and
+// bytes [496, 656) of the token (the last latent bytes, the four scales and
+// both RoPE halves; 160 bytes keeps every group of four rows 128-byte
+// aligned in shared memory).
+constexpr int kTailX = 496;
+constexpr int kTailBytes = 160;
+constexpr int kRawSparseBytes = kRawLatBytes + kPage * kTailBytes;  // 26624
+constexpr int kRawStageBytes = kRawSparseBytes > kRawBytes ? kRawSparseBytes : kRawBytes;
 #ifndef MLA_FP8_RAW_STAGES
 #define MLA_FP8_RAW_STAGES 2
 #endif
@@ -80,6 +88,7 @@ constexpr int kRawBytes = kRawLatBytes + kRawScaleBytes + kRawRopeBytes;  // 215
 #ifndef MLA_BF16_XBUFFERS
 #define MLA_BF16_XBUFFERS 2
 #endif
+
 constexpr int kRawStages = MLA_FP8_RAW_STAGES;
 // Exchange message per tile: fp16 factors [8 chunks of 8 tokens][128 rows][16 B]
 // + the fp32 reference of every row.
@@ -99,6 +108,13 @@ constexpr int kRegCtl = 64;
 constexpr int kRegSoftmax = 176;
 constexpr int kRegDq = 96;
 constexpr int kRegTail = 64;
+// The sparse decode's control warpgroup runs the whole-warp gather (index
+// and block-table reads, row shuffles): control 80, dequant 80.
+constexpr int kRegCtlSparse = 80;
+constexpr int kRegDqSparse = 80;
+constexpr int kRegTailSparse = 80;
+static_assert(kRegCtlSparse + 2 * kRegSoftmax + (kDqWarps / 4) * kRegDqSparse <= (3 + kDqWarps / 4) * kRegLaunchFp8,
+              "register split exceeds the launch budget");
 static_assert(kRegCtl + 2 * kRegSoftmax + (kDqWarps / 4) * kRegDq <= (3 + kDqWarps / 4) * kRegLaunchFp8,
               "register split exceeds the launch budget");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: the lazy reference moves by more than a factor 256
@@ -129,7 +145,7 @@ struct Cfg {
   static constexpr int kXOffset = kStages * kStageBytes;
   static constexpr int kRawOffset = kXOffset + kXBuffers * kXBufBytes;
   // Q's RoPE half-slice (128 rows x 32 dims bf16, SW64 K-major) is an SS operand
-  static constexpr int kQRopeOffset = kRawOffset + (kFp8 ? kRawStages * kRawBytes : 0);
+  static constexpr int kQRopeOffset = kRawOffset + (kFp8 ? kRawStages * kRawStageBytes : 0);
   // [wg][row] fp32: each warpgroup's latest lazy reference; [row] the
   // combined reference of the last consumed tile; [wg][row] the row-sum parts
   // at the item's final scale.  Then barriers, the abort flag, the tensor-
@@ -137,7 +153,11 @@ struct Cfg {
   static constexpr int kRefSlotOffset = kQRopeOffset + kRows * 64;
   static constexpr int kCombSlotOffset = kRefSlotOffset + 2 * kRows * 4;
   static constexpr int kEpiOffset = kCombSlotOffset + kRows * 4;
-  static constexpr int kBarOffset = kEpiOffset + 2 * kRows * 4;
+  // Sparse decode: the validity mask of each raw stage and of each bf16
+  // stage (bit t: token t of the tile is a key).
+  static constexpr int kRawMaskOffset = kEpiOffset + 2 * kRows * 4;
+  static constexpr int kStageMaskOffset = kRawMaskOffset + 8 * kRawStages;
+  static constexpr int kBarOffset = kStageMaskOffset + 8 * kStages;
   // The dynamic shared memory base is 1024-byte aligned (the driver reserves
   // the first 1 KB of the window); the kernel checks it at entry.
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16;
@@ -223,12 +243,19 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float sc, uint32_t (&
   }
 }
 
-template <bool kFp8>
+// kSparse (FP8 only): each unit (a query token) attends to the tokens its
+// index list names instead of a page range; the producer gathers them with
+// per-token bulk copies and a per-tile validity mask replaces the length mask.
+template <bool kFp8, bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_c, const DecodeParams p) {
   using namespace dk;
   using C = Cfg<kFp8>;
+  static_assert(!kSparse || kFp8, "the sparse decode reads the 656-byte FP8 cache");
+  constexpr int kCtlRegs = kSparse ? kRegCtlSparse : kRegCtl;
+  constexpr int kDqRegs = kSparse ? kRegDqSparse : kRegDq;
+  constexpr int kTailRegs = kSparse ? kRegTailSparse : kRegTail;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   TRACE(kTraceCta, 0, 0);
@@ -288,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
+  if (!kSparse && warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
     if (kFp8) tma_prefetch_desc(&tm_c);
@@ -309,7 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     const size_t nthr = static_cast<size_t>(gridDim.x) * blockDim.x;
     const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const size_t qbytes = static_cast<size_t>(p.batch) * p.M * (kDqk * 2);
-    const size_t btbytes = static_cast<size_t>(p.batch) * p.max_pages * 4;
+    const size_t btbytes = static_cast<size_t>(p.req_batch) * p.max_pages * 4;
     const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q);
     const uint8_t* btb = reinterpret_cast<const uint8_t*>(p.block_table);
     for (size_t o = tid * 128; o < qbytes; o += nthr * 128) prefetch_l2_line(qb + o);
@@ -343,8 +370,105 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
   // tail.  (An increase anywhere else could take registers that a softmax
   // warpgroup still waits for: setmaxnreg.inc blocks until the pool can pay.)
   if (warp < 4) {
-    if constexpr (kFp8) setmaxnreg_dec<kRegCtl>();
-  if (warp == 0) {
+    if constexpr (kFp8) setmaxnreg_dec<kCtlRegs>();
+  if (kSparse && warp == 0) {
+    // ------------------------------------------------------------------ sparse gather (whole warp)
+    // Tile j of an item is entries [64 j, 64 j + 64) of the unit's index
+    // list.  Lane l resolves entries l and l + 32: it reads the position,
+    // checks it against the request's length and maps it through the block
+    // table to a row of the cache (viewed as [num_blocks * 64, 656] bytes).
+    // These reads run one tile ahead of the copies.  The copies are TMA
+    // gathers of four rows: lanes 0-15 bring the latent halves of tokens
+    // 4l .. 4l + 3 (256 bytes each), lanes 16-31 their tails (bytes 496-655).
+    // Entries that are not keys (padding, positions outside [0, L), pages that
+    // map outside the cache, which are also reported) fetch row 0 instead and
+    // keep their bit in the stage's mask clear; the dequant writes zeros for
+    // them and the softmax masks their logits.
+    uint64_t* raw_mask = reinterpret_cast<uint64_t*>(sbase + C::kRawMaskOffset);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int it = it_begin; it < it_end && ok; ++it) {
+      const int vb = items[4 * it], p0 = items[4 * it + 1], p1 = items[4 * it + 2];
+      const int u = vb / p.row_tiles;
+      const int req = u / p.req_div;
+      const int L = p.seqlens[req];
+      const int32_t* bt = p.block_table + static_cast<size_t>(req) * p.max_pages;
+      const int32_t* list = p.indices + static_cast<size_t>(u) * p.topk;
+      if (lane == 0 && rank == 0 && p1 > p0) {
+        const int row0 = (vb - u * p.row_tiles) * kRows;
+        const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q) + (static_cast<size_t>(u) * p.M + row0) * (kDqk * 2);
+        const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.M - row0)) * (kDqk * 2);
+        for (uint32_t o = 0; o < bytes; o += 16384u) prefetch_l2_bulk(qb + o, min(16384u, bytes - o));
+      }
+      // rows (-1: not a key) of entries lane and lane + 32 of tile pg
+      auto resolve = [&](int pg, int (&row)[2]) {
+        int pos[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int e = pg * kPage + lane + 32 * k;
+          pos[k] = e < p.topk ? list[e] : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          row[k] = -1;
+          if (pos[k] >= 0 && pos[k] < L) {
+            const int pgi = pos[k] / kPage;
+            const long long blk = pgi < p.max_pages ? bt[pgi] : -1;
+            if (blk < 0 || blk >= p.num_blocks) report_status(p.status, kStatusBadBlock);
+            else row[k] = static_cast<int>(blk) * kPage + pos[k] % kPage;
+          }
+        }
+      };
+      int cur[2], nxt[2] = {-1, -1};
+      if (p1 > p0) resolve(p0, cur);
+      for (int pg = p0; pg < p1; ++pg, ++g) {
+        const uint32_t st = g % kRawStages;
+        if (lane == 0) TRACE(kTraceProducer, g, 0);
+        if (pg + 1 < p1) resolve(pg + 1, nxt);  // its loads overlap the wait below
+        int waited = 1;
+        if (lane == 0 && g >= static_cast<uint32_t>(kRawStages))
+          waited = mbar_wait(BAR(C::kRawEmpty + st), ((g / kRawStages) & 1u) ^ 1u, abort_flag, p.timeout_ns);
+        waited = __shfl_sync(0xffffffffu, waited, 0);
+        if (!waited) {
+          if (lane == 0) raise_abort(p, abort_flag);
+          ok = false;
+          break;
+        }
+        const uint32_t m0 = __ballot_sync(0xffffffffu, cur[0] >= 0), m1 = __ballot_sync(0xffffffffu, cur[1] >= 0);
+        const uint32_t fb = BAR(C::kRawFull + st);
+        if (lane == 0) {
+          raw_mask[st] = (static_cast<uint64_t>(m1) << 32) | m0;
+          mbar_arrive_expect_tx(fb, kRawSparseBytes);
+        }
+        __syncwarp();
+        // rows of tokens 4q .. 4q + 3, q = lane % 16: token t sits in lane
+        // t % 32, slot t / 32
+        const int q4 = lane & 15;
+        int rows[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = 4 * q4 + i;
+          const int r0 = __shfl_sync(0xffffffffu, cur[0], t & 31);
+          const int r1 = __shfl_sync(0xffffffffu, cur[1], t & 31);
+          const int rr = t < 32 ? r0 : r1;
+          rows[i] = rr < 0 ? 0 : rr;
+        }
+        const uint32_t dst = rawbuf0 + st * kRawStageBytes;
+        if (lane < 16)
+          tma_gather4(dst + q4 * 4 * 256, &tm_a, fb, static_cast<int>(rank) * 256, rows[0], rows[1], rows[2], rows[3]);
+        else
+          tma_gather4(dst + kRawLatBytes + q4 * 4 * kTailBytes, &tm_b, fb, kTailX, rows[0], rows[1], rows[2],
+                      rows[3]);
+        cur[0] = nxt[0];
+        cur[1] = nxt[1];
+        if (lane == 0) TRACE(kTraceProducer, g, 1);
+      }
+    }
+    // Never leave a copy landing in shared memory after the CTA exits.
+    if (lane == 0)
+      for (uint32_t k = (g > static_cast<uint32_t>(kRawStages) ? g - kRawStages : 0u); k < g; ++k)
+        mbar_wait(BAR(C::kRawFull + k % kRawStages), (k / kRawStages) & 1u, &g_never_abort, 100000000ull);
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // BF16: page halves straight into the MMA stages.  FP8: raw bytes into
@@ -380,6 +504,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         for (int pg = p0; pg < p1; ++pg, ++g) {
           const uint32_t st = g % nst;
           TRACE(kTraceProducer, g, 0);
+          // BF16, the CTA's first item: page 0 goes out with the Q loads, the
+          // rest of the prefetch only once Q is in tensor memory.  At a
+          // kernel's start every CTA loads Q and fills all its stages at
+          // once; served in that order, Q and page 0 arrive first and the
+          // tensor pipe starts earlier while the other pages stream in behind
+          // them (uniform batch 103.4 -> 101.4 us).  FP8 keeps its raw stages
+          // filling from the start: its dequant warps need them first (2%
+          // slower with the same order).
+          if (!kFp8 && it == it_begin && pg == p0 + 1 &&
+              !mbar_wait(BAR(C::kQReady), 0, abort_flag, p.timeout_ns)) {
+            raise_abort(p, abort_flag);
+            ok = false;
+            break;
+          }
           if (g >= static_cast<uint32_t>(nst) &&
               !mbar_wait(BAR(empty0 + st), ((g / nst) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
             raise_abort(p, abort_flag);
@@ -401,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           const int y = static_cast<int>(phys) * kPage;
           const uint32_t fb = BAR(full0 + st);
           if constexpr (kFp8) {
-            const uint32_t dst = rawbuf0 + st * kRawBytes;
+            const uint32_t dst = rawbuf0 + st * kRawStageBytes;
             mbar_arrive_expect_tx(fb, kRawBytes);
             tma_load_2d(dst, &tm_a, fb, static_cast<int>(rank) * 256, y);
             tma_load_2d(dst + kRawLatBytes, &tm_b, fb, 512, y);
@@ -496,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
   }
     __syncwarp();
-    static_assert(kRegCtl == kRegTail, "the control warps stay at their budget for the tail");
+    static_assert(kCtlRegs == kTailRegs, "the control warps stay at their budget for the tail");
   } else if (warp < 4 + kSoftmaxWarps) {
     // ------------------------------------------------------------------ softmax / epilogue
     if constexpr (kFp8) setmaxnreg_inc<kRegSoftmax>();
@@ -525,7 +663,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       const int b = vb / p.row_tiles, row0 = (vb - b * p.row_tiles) * kRows;
       const bool row_ok = row0 + r < p.M;   // this thread's row exists in the request
       const int qi = (row0 + r) / p.h_q;    // its query token
-      const int L = p.seqlens[b];
+      const int L = p.seqlens[b / p.req_div];
       const int n = p1 - p0;
       const size_t orow = static_cast<size_t>(b) * p.M + row0 + r;
       if (n <= 0) {
@@ -616,7 +754,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (lane == 0) mbar_arrive(BAR(C::kSFree));
         if (wt == 0) TRACE(kTraceSoftmax, gg, 2);
         const int tok0 = pg * kPage;
-        const bool full_tile = tok0 + kPage <= vis_all;
+        // Sparse decode: the tile's validity mask, written by the dequant warps
+        // before they completed the stage's full barrier; acquiring that
+        // (already completed) phase makes the write visible here.  The stage
+        // is not refilled before this tile's P*V, so the mask stays put.
+        uint64_t vmask = ~0ull;
+        if constexpr (kSparse) {
+          const uint32_t st = gg % kStages;
+          if (!warp_wait(BAR(C::kFull + st), (gg / kStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          vmask = *reinterpret_cast<const volatile uint64_t*>(sbase + C::kStageMaskOffset + 8 * st);
+        }
+        const bool full_tile = kSparse ? (vmask == ~0ull) : (tok0 + kPage <= vis_all);
         float e[64];
         float tmax;
         {
@@ -635,7 +783,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
             tmax = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])) * c_abs;
           } else {
 #pragma unroll
-            for (int t = 0; t < 64; ++t) e[t] = (tok0 + t < vis) ? __uint_as_float(s[t]) * c_log2 : -CUDART_INF_F;
+            for (int t = 0; t < 64; ++t) {
+              const bool key = kSparse ? ((vmask >> t) & 1ull) != 0 : (tok0 + t < vis);
+              e[t] = key ? __uint_as_float(s[t]) * c_log2 : -CUDART_INF_F;
+            }
 #pragma unroll
             for (int t = 0; t < 32; ++t) a[t & 3] = fmax3(a[t & 3], e[2 * t], e[2 * t + 1]);
             tmax = fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
@@ -878,10 +1029,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
     if (!ok) raise_abort(p, abort_flag);
     __syncwarp();
-    if constexpr (kFp8) setmaxnreg_dec<kRegTail>();
+    if constexpr (kFp8) setmaxnreg_dec<kTailRegs>();
   } else if (kFp8) {
     // ------------------------------------------------------------------ FP8 dequant (warps 12-15)
-    setmaxnreg_dec<kRegDq>();
+    setmaxnreg_dec<kDqRegs>();
     // Raw 656-byte tokens -> this CTA's bf16 page half, in the same swizzled
     // layout the BF16 path gets from TMA.  Thread dt handles 16-code units
     // u = dt + 128 k: token u / 16, codes 16 (u % 16) .. +16 of the CTA's 256.
@@ -891,7 +1042,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     bool ok = true;
     for (int it = it_begin; it < it_end && ok; ++it) {
       const int p0 = items[4 * it + 1], p1 = items[4 * it + 2];
-      const int L = p.seqlens[items[4 * it] / p.row_tiles];
+      const int L = p.seqlens[items[4 * it] / p.row_tiles / p.req_div];
       const int last_page = (L - 1) / kPage;
       for (int pg = p0; pg < p1; ++pg, ++g) {
         const uint32_t rs = g % kRawStages, st = g % kStages;
@@ -901,19 +1052,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         if (g >= static_cast<uint32_t>(kStages) &&
             !warp_wait(BAR(C::kEmpty + st), ((g / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         if (dt == 0) TRACE(kTraceDequant, g, 2);
+        // Token t of the tile is a key: t below the request's length on its
+        // last page, or (sparse) its bit in the mask the gather wrote.
         const int valid = (pg == last_page) ? L - pg * kPage : kPage;
-        const uint8_t* rlat = sbase + C::kRawOffset + rs * kRawBytes;
-        const uint8_t* rscale = rlat + kRawLatBytes;
-        const uint8_t* rrope = rscale + kRawScaleBytes;
+        uint64_t tmask = 0;
+        if constexpr (kSparse) tmask = *reinterpret_cast<const volatile uint64_t*>(sbase + C::kRawMaskOffset + 8 * rs);
+        const uint8_t* rlat = sbase + C::kRawOffset + rs * kRawStageBytes;
+        // where token t's scales and this CTA's RoPE half are: the dense copy
+        // lays them out as [64][16] and [64][64]; the sparse gather brings
+        // bytes 496-655 of each token as one 160-byte row
+        const uint8_t* rscale = rlat + kRawLatBytes + (kSparse ? 512 - kTailX : 0);
+        const uint8_t* rrope = kSparse ? rlat + kRawLatBytes + (528 - kTailX) + 64 * static_cast<int>(rank)
+                                       : rlat + kRawLatBytes + kRawScaleBytes;
+        constexpr int kScaleStride = kSparse ? kTailBytes : 16;
+        constexpr int kRopeStride = kSparse ? kTailBytes : 64;
         uint8_t* dst = sbase + st * kStageBytes;
 #pragma unroll 2
         for (int k = 0; k < 1024 / kDqThreads; ++k) {
           const int u = dt + kDqThreads * k;
           const int t = u >> 4, g16 = u & 15;
           uint32_t w[8];
-          if (t < valid) {
+          if (kSparse ? ((tmask >> t) & 1ull) != 0 : t < valid) {
             const uint4 codes = *reinterpret_cast<const uint4*>(rlat + t * 256 + g16 * 16);
-            const float sc = *reinterpret_cast<const float*>(rscale + t * 16 + 4 * (2 * static_cast<int>(rank) + (g16 >> 3)));
+            const float sc =
+                *reinterpret_cast<const float*>(rscale + t * kScaleStride + 4 * (2 * static_cast<int>(rank) + (g16 >> 3)));
             dequant16(codes, sc, w);
           } else {
 #pragma unroll
@@ -929,9 +1091,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           const int u = dt + kDqThreads * k;
           const int t = u >> 2, w4 = u & 3;
           uint4 v = make_uint4(0, 0, 0, 0);
-          if (t < valid) v = *reinterpret_cast<const uint4*>(rrope + t * 64 + w4 * 16);
+          if (kSparse ? ((tmask >> t) & 1ull) != 0 : t < valid)
+            v = *reinterpret_cast<const uint4*>(rrope + t * kRopeStride + w4 * 16);
           *reinterpret_cast<uint4*>(dst + 4 * kChunkBytes + t * 64 + ((w4 ^ ((t >> 1) & 3)) << 4)) = v;
         }
+        // sparse: the mask goes with the bf16 stage to the softmax warps
+        if (kSparse && dt == 0) *reinterpret_cast<volatile uint64_t*>(sbase + C::kStageMaskOffset + 8 * st) = tmask;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -943,7 +1108,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     }
     if (!ok) raise_abort(p, abort_flag);
     __syncwarp();
-    setmaxnreg_dec<kRegTail>();
+    if constexpr (kDqRegs != kTailRegs) setmaxnreg_dec<kTailRegs>();
   }
 
   tc_fence_before();
@@ -978,7 +1143,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 #undef BAR
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kSparse>
 static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_c,
                                  const DecodeParams& p, int num_parts, cudaStream_t stream) {
   using C = dk::Cfg<kFp8>;
@@ -992,7 +1157,8 @@ static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_
   if (e != cudaSuccess) return e;
   const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
   if (bit == 0 || (attr_done.load(std::memory_order_acquire) & bit) == 0) {
-    e = cudaFuncSetAttribute(decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(decode_kernel<kFp8, kSparse>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
@@ -1009,17 +1175,24 @@ static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<kFp8>, tm_a, tm_b, tm_c, p);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<kFp8, kSparse>, tm_a, tm_b, tm_c, p);
 }
 
 cudaError_t launch_decode_bf16(const CUtensorMap& tm_lat, const CUtensorMap& tm_rope, const DecodeParams& p,
                                int num_parts, cudaStream_t stream) {
-  return launch_decode<false>(tm_lat, tm_rope, tm_rope, p, num_parts, stream);
+  return launch_decode<false, false>(tm_lat, tm_rope, tm_rope, p, num_parts, stream);
 }
 
 cudaError_t launch_decode_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_scale, const CUtensorMap& tm_rope,
                               const DecodeParams& p, int num_parts, cudaStream_t stream) {
-  return launch_decode<true>(tm_lat, tm_scale, tm_rope, p, num_parts, stream);
+  return launch_decode<true, false>(tm_lat, tm_scale, tm_rope, p, num_parts, stream);
+}
+
+// The sparse decode gathers rows: tm_lat has a (256 x 1)-byte box, tm_tail a
+// (160 x 1)-byte one, both over the cache viewed as [num_blocks * 64, 656].
+cudaError_t launch_decode_sparse_fp8(const CUtensorMap& tm_lat, const CUtensorMap& tm_tail, const DecodeParams& p,
+                                     int num_parts, cudaStream_t stream) {
+  return launch_decode<true, true>(tm_lat, tm_tail, tm_tail, p, num_parts, stream);
 }
 
 }  // namespace mla

@@ -20,6 +20,8 @@
 // Requests with more than 128 query rows: everything above is over virtual
 // requests v = b * row_tiles + tile, each with the length of request b, so
 // "batch" below is the virtual batch and v's length is seqlens[v / row_tiles].
+// With seqlens == nullptr every virtual request has the length uniform_len
+// (the sparse decode: each query token attends to a list of topk entries).
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -69,9 +71,9 @@ __device__ __forceinline__ int block_max(int v, int* warp_sums) {
   return m;
 }
 
-__global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
-                                                                int rtiles, int parts, int overhead,
-                                                                int32_t* __restrict__ sched,
+__global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* __restrict__ seqlens,
+                                                                int uniform_len, int batch, int rtiles, int parts,
+                                                                int overhead, int32_t* __restrict__ sched,
                                                                 int32_t* __restrict__ num_splits) {
   // the decode kernel may begin launching (it waits for this grid to complete)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -87,14 +89,14 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
   // 1. cost prefix
   int local = 0;
   for (int b = b0; b < b1; ++b) {
-    int L = max(seqlens[b / rtiles], 0);
+    int L = (seqlens ? max(seqlens[b / rtiles], 0) : uniform_len);
     local += (L + kPage - 1) / kPage + overhead;
   }
   int T;
   int run = block_exclusive_scan(local, warp_sums, &T);
   for (int b = b0; b < b1; ++b) {
     C[b] = run;
-    int L = max(seqlens[b / rtiles], 0);
+    int L = (seqlens ? max(seqlens[b / rtiles], 0) : uniform_len);
     run += (L + kPage - 1) / kPage + overhead;
   }
   if (threadIdx.x == 0) C[batch] = T;
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
     int32_t* part_first = sched + kSchedHeader;
     int32_t* items = sched + sched_items_offset(parts);
     for (int b = b0; b < b1; ++b) {
-      const int L = max(seqlens[b / rtiles], 0);
+      const int L = (seqlens ? max(seqlens[b / rtiles], 0) : uniform_len);
       items[4 * b + 0] = b;
       items[4 * b + 1] = 0;
       items[4 * b + 2] = (L + kPage - 1) / kPage;
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
   int nsplit_req;
   int split_pos = block_exclusive_scan(local, warp_sums, &nsplit_req);
   for (int b = b0; b < b1; ++b) {
-    const int L = max(seqlens[b / rtiles], 0);
+    const int L = (seqlens ? max(seqlens[b / rtiles], 0) : uniform_len);
     const int n = (L + kPage - 1) / kPage;
     const int cb = C[b], cost = C[b + 1] - C[b];
     const int k0 = cb / t, k1 = (C[b + 1] - 1) / t;
@@ -206,9 +208,10 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
   }
 }
 
-// `batch` is the virtual batch (requests * rtiles).
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int rtiles, int parts, int32_t* sched,
-                            int32_t* num_splits, cudaStream_t stream) {
+// `batch` is the virtual batch (requests * rtiles); seqlens == nullptr gives
+// every virtual request the length uniform_len.
+cudaError_t launch_metadata(const int32_t* seqlens, int uniform_len, int batch, int rtiles, int parts,
+                            int32_t* sched, int32_t* num_splits, cudaStream_t stream) {
   const size_t smem = 2ull * (batch + 1) * sizeof(int);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -218,7 +221,7 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int rtiles, int p
   // one request per thread up to 1024 requests (whole warps): small batches
   // sync fewer warps in the block scans
   const int threads = batch >= kMetaThreads ? kMetaThreads : ((batch + 31) / 32) * 32;
-  metadata_kernel<<<1, threads > 0 ? threads : 32, smem, stream>>>(seqlens, batch, rtiles, parts,
+  metadata_kernel<<<1, threads > 0 ? threads : 32, smem, stream>>>(seqlens, uniform_len, batch, rtiles, parts,
                                                                   kSplitOverheadPages, sched, num_splits);
   return cudaGetLastError();
 }

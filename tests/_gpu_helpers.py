@@ -87,6 +87,48 @@ def oracle_chunked(case, dequant_bf16=False, chunk=16):
     return out, lse
 
 
+def run_gpu_sparse(case, indices, num_sm_parts=None, workspace=None):
+    """The sparse decode through the C ABI -> (out, lse, status) as float64 numpy."""
+    import mla_paged_kv_04_b200 as mla
+    dev = torch.device("cuda")
+    q = case["q"].to(dev)
+    kv = case["kv_cache"].to(dev)
+    bt = case["block_table"].to(dev)
+    L = case["cache_seqlens"].to(dev)
+    idx = indices.to(dev)
+    B, s_q, h_q, _ = q.shape
+    parts = mla.mla_default_num_sm_parts() if num_sm_parts is None else num_sm_parts
+    sched, ns = mla.mla_get_sparse_metadata(B, s_q, h_q, idx.shape[2], parts, device=dev)
+    if workspace is None:
+        workspace = torch.zeros(mla.mla_sparse_workspace_size(B, s_q, h_q, parts), dtype=torch.uint8, device=dev)
+    out = torch.empty((B, s_q, h_q, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    mla.mla_sparse_decode_fwd(q, kv, bt, L, idx, case["softmax_scale"], sched, ns, parts, out, lse, workspace)
+    status = mla.mla_last_device_status(workspace)
+    return out.float().cpu().double().numpy(), lse.cpu().double().numpy(), status
+
+
+def oracle_sparse(case, indices, dequant_bf16=False, chunk=16):
+    """Sparse-decode oracle outputs for every request, a few requests at a time
+    on compact copies of their pages."""
+    B = case["batch"]
+    idx = indices.cpu().numpy()
+    out = np.zeros((B, case["s_q"], case["h_q"], 512))
+    lse = np.full((B, case["s_q"], case["h_q"]), -np.inf)
+    for b0 in range(0, B, chunk):
+        reqs = list(range(b0, min(B, b0 + chunk)))
+        a = W.oracle_arrays_for(case, reqs)
+        if dequant_bf16 and a["fmt"] == "fp8_656":
+            kv = fp8_cache_as_bf16(torch.from_numpy(a["kv_cache"]))
+            a["kv_cache"] = kv.view(torch.int16).numpy().view(np.uint16)
+            a["fmt"] = "bf16"
+        o, l = oracle.mla_sparse_decode(a["q_bits"][reqs], a["kv_cache"], a["fmt"], a["block_table"][reqs],
+                                        a["cache_seqlens"][reqs], idx[reqs], a["softmax_scale"])
+        out[b0:b0 + len(reqs)] = o
+        lse[b0:b0 + len(reqs)] = l
+    return out, lse
+
+
 def check(out, lse, ref_out, ref_lse, what=""):
     """Element-wise comparison; -inf lse must match exactly (empty rows)."""
     err = np.abs(out - ref_out)

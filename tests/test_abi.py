@@ -213,3 +213,14 @@ def test_binding_rejects_host_tensors_before_the_c_abi():
         mla.mla_kv_append(torch.zeros((B, 1, 576), dtype=torch.bfloat16), kv, "bf16", bt, L, ws)
     with pytest.raises(ValueError):
         mla.mla_get_metadata(L, 1, 16, 74)
+
+
+def test_binding_device_check_resolves_an_unindexed_cuda_device(monkeypatch):
+    # torch.device("cuda") names the current device, while tensors report
+    # cuda:<index>; the check compares against the resolved index (and still
+    # rejects a host tensor, naming that device).
+    import torch
+    import mla_paged_kv_04_b200 as mla
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="cuda:0"):
+        mla._on_device(torch.device("cuda"), t=torch.zeros(4))

@@ -57,3 +57,12 @@ def test_reference_line_keys():
     assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1 and cpu["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_sparse_work_counts_valid_entries_only():
+    w = W.Workload("s", 2, 1, 16, (1, 1), fmt="fp8_656", topk=4)
+    L = np.array([10, 3])
+    idx = np.array([[[0, 9, -1, 10]], [[2, 2, 5, -7]]])  # valid: 2 + 2
+    work = bench.sparse_work(w, L, idx)
+    assert work["flops"] == 2 * (576 + 512) * 16 * 4
+    assert work["bytes"] == 656 * 4 + 2 * 16 * (1152 + 1024 + 4) + 4 * idx.size + 4 * 4 + 4 * 2

@@ -23,6 +23,11 @@ Recipe (all draws from one torch.Generator seeded with `seed`, default 0):
      a group with amax 0 gets scale 0 and codes 0.  RoPE slice N(0,1) bf16.
   5. Poison (default on): tail slots of each request's last page and all
      spare blocks are filled with NaN/Inf patterns; they must never be read.
+  6. Sparse workloads (topk > 0): for every (request b, query token i) an
+     index list of topk positions: a uniformly random set of topk distinct
+     positions of [0, L_b) in increasing order (the form a top-k selector
+     returns), or, when L_b < topk, every position followed by -1 padding.
+     The selector itself is not modelled (it needs trained weights).
 """
 
 from __future__ import annotations
@@ -50,6 +55,7 @@ class Workload:
     causal: bool = False
     seed: int = 0
     spare_frac: float = 0.05
+    topk: int = 0  # > 0: a sparse decode with index lists of topk entries
 
     @property
     def softmax_scale(self) -> float:
@@ -59,7 +65,7 @@ class Workload:
         lo, hi = self.seqlen
         L = f"{lo}" if lo == hi else f"U[{lo},{hi}]"
         return (f"{self.name}: b={self.batch} s_q={self.s_q} h_q={self.h_q} L={L} "
-                f"{self.fmt}{' causal' if self.causal else ''}")
+                f"{self.fmt}{' causal' if self.causal else ''}{f' topk={self.topk}' if self.topk else ''}")
 
 
 WORKLOADS = {
@@ -68,8 +74,47 @@ WORKLOADS = {
     "varlen_spec_bf16": Workload("varlen_spec_bf16", 128, 2, 64, (1, 8192), causal=True),
     "fp8_656": Workload("fp8_656", 128, 1, 128, (16384, 32768), fmt="fp8_656"),
     "long_ctx_bf16": Workload("long_ctx_bf16", 8, 1, 128, (131072, 131072)),
+    # the sparse decode over the FP8 workload's cache: 2048 listed tokens per query
+    "sparse_fp8": Workload("sparse_fp8", 128, 1, 128, (16384, 32768), fmt="fp8_656", topk=2048),
 }
 ORDER = ["tiny", "uniform_bf16", "varlen_spec_bf16", "fp8_656", "long_ctx_bf16"]
+SPARSE_ORDER = ["sparse_fp8"]
+
+
+def make_sparse_indices(cache_seqlens, s_q: int, topk: int, seed: int = 0, device="cpu", pad: int = 0,
+                        dup: int = 0, oob: int = 0):
+    """Index lists int32 [batch, s_q, topk] (recipe step 6).
+
+    Optional edge cases for tests, per list: `dup` entries overwritten with a
+    repeat of another entry, `pad` with -1, `oob` with positions >= L_b.
+    """
+    gen = torch.Generator()
+    gen.manual_seed(seed + 12345)
+    L = [int(x) for x in torch.as_tensor(cache_seqlens).cpu().tolist()]
+    B = len(L)
+    idx = torch.full((B, s_q, topk), -1, dtype=torch.int32)
+    for b in range(B):
+        for i in range(s_q):
+            n = min(topk, L[b])
+            if n > 0:
+                sel = torch.randperm(L[b], generator=gen)[:n] if L[b] > topk else torch.arange(L[b])
+                idx[b, i, :n] = torch.sort(sel.to(torch.int32)).values
+            row = idx[b, i]
+            slots = torch.randperm(topk, generator=gen)
+            k = 0
+            for _ in range(min(dup, n)):
+                src = int(torch.randint(0, n, (1,), generator=gen))
+                row[int(slots[k])] = row[src] if int(row[src]) >= 0 else 0
+                k += 1
+            for _ in range(pad):
+                if k < topk:
+                    row[int(slots[k])] = -1
+                    k += 1
+            for _ in range(oob):
+                if k < topk:
+                    row[int(slots[k])] = L[b] + int(torch.randint(0, 1000, (1,), generator=gen))
+                    k += 1
+    return idx.to(device)
 
 # NaN / Inf bit patterns used as poison.
 _BF16_POISON = (0x7FC0, 0xFF80, 0xFFFF, 0x7F80)
@@ -157,11 +202,14 @@ def make_case(w: Workload, seed: int | None = None, device="cpu", poison: bool =
     if poison:
         _poison(kv, w.fmt, bt, L, spare_blocks)
 
-    return dict(
+    case = dict(
         workload=w, q=q, kv_cache=kv, block_table=bt.to(device), cache_seqlens=L.to(device),
         softmax_scale=w.softmax_scale, causal=w.causal, fmt=w.fmt, num_blocks=num_blocks,
         s_q=w.s_q, h_q=w.h_q, batch=B,
     )
+    if w.topk:
+        case["indices"] = make_sparse_indices(L, w.s_q, w.topk, seed=seed, device=device)
+    return case
 
 
 def _poison(kv, fmt, bt, L, spare_blocks):
