@@ -50,6 +50,10 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "MLA decode TFLOPS & effective HBM GB/s on 1 B200 (frac of roofline)"
+# the arithmetic the tensor cores run on for each cache format
+MMA = {"bf16": "bf16 operands, fp32 accumulation",
+       "fp8_656": "bf16 operands (FP8 cache dequantised to bf16 in shared memory), fp32 accumulation"}
+DTYPE = {"bf16": "bf16", "fp8_656": "bf16"}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -562,7 +566,7 @@ def measure_workload(w: W.Workload, args, world, rank, dev, peaks, cpu_budget: f
         "unit": "TFLOP/s", "gbs": aggregate_rate(work["bytes"], ms_per_step, n) / 1e9,
         "ms_per_step": ms_per_step, "metadata_ms": statistics.median(meta_ms),
         "config": {"workload": w.describe(), "batch": B, "s_q": w.s_q, "h_q": w.h_q, "seqlen": list(w.seqlen),
-                   "kv_format": w.fmt, "causal": w.causal, "num_sm_parts": parts},
+                   "kv_format": w.fmt, "causal": w.causal, "num_sm_parts": parts, "mma": MMA[w.fmt]},
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": {"value": n * work["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "gbs": n * work["bytes"] / (e2e_ms * 1e-3) / 1e9,
@@ -602,9 +606,8 @@ def run_cuda(args, world, rank, local):
     line = {
         "metric": METRIC, "value": rec["value"], "unit": rec["unit"], "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": DTYPE[head.fmt], "data": "synthetic",
         "config": dict(rec["config"], **{
-            "mma": "bf16 operands (FP8 cache dequantised in shared memory), fp32 accumulation",
             "launch": "each timed step replays a CUDA graph of the public calls (schedule, decode, combine)",
             "l2": "flushed before every timed step and every roofline rep (256 MiB write)",
             "parallelism": f"replicas x{n} (independent request batches)"}),

@@ -244,8 +244,8 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float sc, uint32_t (&
 }
 
 // kSparse (FP8 only): each unit (a query token) attends to the tokens its
-// index list names instead of a page range; the producer gathers them with
-// per-token bulk copies and a per-tile validity mask replaces the length mask.
+// index list names instead of a page range; the producer gathers their rows
+// with TMA gathers and a per-tile validity mask replaces the length mask.
 template <bool kFp8, bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,

@@ -97,8 +97,9 @@ def unpack_fp8_656(tokens: np.ndarray) -> np.ndarray:
 
     key[d] = e4m3(byte d) * scale[d // 128]    for d < 512   (R4, R5)
     key[d] = bf16 RoPE value d - 512           for d >= 512
-    The product is formed exactly in float64 (the page's "same dequantised
-    cache" is the exact product; rounding it is the kernel's business).
+    The product is formed exactly in float64; how a kernel rounds it is that
+    kernel's business (the FP8 parity tests additionally feed the oracle the
+    keys rounded the way the kernel rounds them, as a BF16 cache).
     """
     t = np.ascontiguousarray(np.asarray(tokens, dtype=np.uint8))
     assert t.shape[-1] == FP8_TOKEN_BYTES

@@ -125,6 +125,30 @@ def test_fp8_roundtrip_through_generator():
     assert np.all((mags.max(axis=2) == 0x7E) | (scale == 0))
 
 
+def test_bf16_dequant_mirror_is_one_rounding_of_the_exact_keys():
+    """The FP8 parity tests feed the oracle the cache the CUDA path computes on
+    (reading R8): latent dims bf16(fp32(e4m3) * fp32(scale)), RoPE as stored.
+    Pinned against the exact products: within one bf16 rounding (2^-8
+    relative, plus the fp32 product's 2^-24) of them; equal to them when the scale is a power of two (an
+    e4m3 code times a power of two is a bf16 number); the RoPE dims untouched."""
+    from _gpu_helpers import fp8_cache_as_bf16
+    g = torch.Generator().manual_seed(8)
+    n = 640
+    lat = (torch.randn(n, 512, generator=g) * torch.tensor([0.3, 1.0, 7.0, 50.0]).repeat_interleave(128))
+    rope = torch.randn(n, 64, generator=g).to(torch.bfloat16)
+    packed = W.quantize_fp8_656(lat.to(torch.bfloat16), rope)
+    pk = packed.clone()
+    pk[:64, 512:528] = torch.full((64, 4), 0.0625).view(torch.uint8).reshape(64, 16)  # tokens 0-63: scale 2^-4
+    mirror = fp8_cache_as_bf16(pk.view(n // 64, 64, 656)).reshape(n, 576).double().numpy()
+    exact = oracle.unpack_fp8_656(pk.numpy())
+    np.testing.assert_array_equal(mirror[:64], exact[:64])
+    err = np.abs(mirror[64:, :512] - exact[64:, :512])
+    assert np.all(err <= np.abs(exact[64:, :512]) * (2.0 ** -8 + 2.0 ** -23))
+    assert np.all(mirror[64:, :512][exact[64:, :512] == 0] == 0)
+    assert err.max() > 0  # the rounding is really there
+    np.testing.assert_array_equal(mirror[:, 512:], rope.double().numpy())
+
+
 # ---------------------------------------------------------------------------
 # attention pins
 # ---------------------------------------------------------------------------
