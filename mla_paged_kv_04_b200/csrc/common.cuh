@@ -33,16 +33,20 @@ constexpr int kSplitOverheadPages = 4;
 // A schedule that splits requests pays for it outside the page loop: the
 // fp32 partial outputs go to memory and come back in the combine kernel, and
 // a CTA pair that serves two items drains and refills its pipeline in
-// between.  When the batch fits one request per CTA pair, the schedule keeps
-// requests whole unless that makes the longest part longer than the balanced
+// between.  The schedule keeps requests whole (ceil(batch / parts) of them
+// per CTA pair) unless that makes the longest part longer than the balanced
 // cut by more than this many pages.
-constexpr int kSplitPenaltyPages = 16;
+#ifndef MLA_SPLIT_PENALTY_PAGES
+#define MLA_SPLIT_PENALTY_PAGES 16
+#endif
+constexpr int kSplitPenaltyPages = MLA_SPLIT_PENALTY_PAGES;
 
 // Schedule buffer (int32) written by the metadata kernel, over the virtual
 // requests (request, row tile) of the batch:
 //   [0] num_parts  [1] total_items  [2] units per part  [3] virtual batch
 //   (batch * row tiles)  [4] overhead   [5] number of split virtual requests
-//   [6] 1 if whole requests (one per part, no split), else 0  [7] row tiles
+//   [6] 1 if whole requests (ceil(batch / parts) consecutive ones per
+//   part, no split), else 0  [7] row tiles
 //   [8, 8 + num_parts + 1)          first item index of each part
 //   then num_parts ints             ids of the split requests (first [5] valid)
 //   then (16-byte aligned) 4 ints per item: request b, first page, end page, slot

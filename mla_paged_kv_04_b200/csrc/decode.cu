@@ -72,7 +72,6 @@ constexpr int kRawBytes = kRawLatBytes + kRawScaleBytes + kRawRopeBytes;  // 215
 constexpr int kTailX = 496;
 constexpr int kTailBytes = 160;
 constexpr int kRawSparseBytes = kRawLatBytes + kPage * kTailBytes;  // 26624
-constexpr int kRawStageBytes = kRawSparseBytes > kRawBytes ? kRawSparseBytes : kRawBytes;
 #ifndef MLA_FP8_RAW_STAGES
 #define MLA_FP8_RAW_STAGES 2
 #endif
@@ -88,8 +87,20 @@ constexpr int kRawStageBytes = kRawSparseBytes > kRawBytes ? kRawSparseBytes : k
 #ifndef MLA_BF16_XBUFFERS
 #define MLA_BF16_XBUFFERS 2
 #endif
-
-constexpr int kRawStages = MLA_FP8_RAW_STAGES;
+// The sparse decode: the same pipeline depths as the dense FP8 path (four
+// raw stages with two dequantised stages and two exchange buffers, or three
+// raw stages with two dequantised ones, measured 6% slower: a dequantised
+// stage is held from its dequant until P*V has read it, and two of them
+// leave the dequant waiting).
+#ifndef MLA_SPARSE_RAW_STAGES
+#define MLA_SPARSE_RAW_STAGES 2
+#endif
+#ifndef MLA_SPARSE_STAGES
+#define MLA_SPARSE_STAGES 3
+#endif
+#ifndef MLA_SPARSE_XBUFFERS
+#define MLA_SPARSE_XBUFFERS 3
+#endif
 // Exchange message per tile: fp16 factors [8 chunks of 8 tokens][128 rows][16 B]
 // + the fp32 reference of every row.
 constexpr int kXERegionBytes = 8 * kRows * 16;          // 16384
@@ -119,13 +130,17 @@ static_assert(kRegCtl + 2 * kRegSoftmax + (kDqWarps / 4) * kRegDq <= (3 + kDqWar
               "register split exceeds the launch budget");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: the lazy reference moves by more than a factor 256
 
-template <bool kFp8>
+template <bool kFp8, bool kSparse = false>
 struct Cfg {
-  static constexpr int kStages = kFp8 ? MLA_FP8_STAGES : MLA_BF16_STAGES;  // bf16 page-half stages
+  // bf16 page-half stages
+  static constexpr int kStages = kSparse ? MLA_SPARSE_STAGES : kFp8 ? MLA_FP8_STAGES : MLA_BF16_STAGES;
+  // FP8: raw 656-byte-format stages, and the bytes of one
+  static constexpr int kRawStages = kSparse ? MLA_SPARSE_RAW_STAGES : MLA_FP8_RAW_STAGES;
+  static constexpr int kRawStageBytes = kSparse ? kRawSparseBytes : kRawBytes;
   // Pair-exchange receive buffers: tile g uses buffer g % kXBuffers, and the
   // peer writes tile g + kXBuffers's message into it only after this CTA has
   // read tile g's (a remote arrive on the peer's "buffer free" barrier).
-  static constexpr int kXBuffers = kFp8 ? MLA_FP8_XBUFFERS : MLA_BF16_XBUFFERS;
+  static constexpr int kXBuffers = kSparse ? MLA_SPARSE_XBUFFERS : kFp8 ? MLA_FP8_XBUFFERS : MLA_BF16_XBUFFERS;
   static constexpr int kThreads = kFp8 ? 384 + 32 * kDqWarps : 384;
   static constexpr int kFull = 0;
   static constexpr int kEmpty = kFull + kStages;
@@ -251,7 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_c, const DecodeParams p) {
   using namespace dk;
-  using C = Cfg<kFp8>;
+  using C = Cfg<kFp8, kSparse>;
   static_assert(!kSparse || kFp8, "the sparse decode reads the 656-byte FP8 cache");
   constexpr int kCtlRegs = kSparse ? kRegCtlSparse : kRegCtl;
   constexpr int kDqRegs = kSparse ? kRegDqSparse : kRegDq;
@@ -304,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     mbar_init(BAR(C::kCChain), 128);  // every thread of the consuming warpgroup
     mbar_init(BAR(C::kEpi), kSoftmaxWarps * 32);
     for (int i = 0; i < C::kXBuffers; ++i) mbar_init(BAR(C::kXFree + i), 4);  // the peer warpgroup's four warps
-    for (int i = 0; i < kRawStages; ++i) {
+    for (int i = 0; i < C::kRawStages; ++i) {
       mbar_init(BAR(C::kRawFull + i), 1);
       mbar_init(BAR(C::kRawEmpty + i), kDqWarps);
     }
@@ -400,34 +415,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const uint32_t bytes = static_cast<uint32_t>(min(kRows, p.M - row0)) * (kDqk * 2);
         for (uint32_t o = 0; o < bytes; o += 16384u) prefetch_l2_bulk(qb + o, min(16384u, bytes - o));
       }
-      // rows (-1: not a key) of entries lane and lane + 32 of tile pg
-      auto resolve = [&](int pg, int (&row)[2]) {
-        int pos[2];
+      // Each tile's rows take two dependent reads (its list entries, then the
+      // block table): start this item's slice of the list and the request's
+      // block-table row towards L2 now, so that those reads hit L2.  Only
+      // whole 16-byte granules inside each array are prefetched.
+      if (lane == 0 && p1 > p0) {
+        auto prefetch_range = [](const int32_t* first, const int32_t* last) {
+          const uintptr_t a0 = (reinterpret_cast<uintptr_t>(first) + 15u) & ~static_cast<uintptr_t>(15);
+          const uintptr_t a1 = reinterpret_cast<uintptr_t>(last) & ~static_cast<uintptr_t>(15);
+          for (uintptr_t a = a0; a < a1; a += 16384u)
+            prefetch_l2_bulk(reinterpret_cast<const void*>(a), static_cast<uint32_t>(a1 - a < 16384u ? a1 - a : 16384u));
+        };
+        prefetch_range(list + p0 * kPage, list + min(p1 * kPage, p.topk));
+        if (rank == 0) prefetch_range(bt, bt + min((max(L, 0) + kPage - 1) / kPage, p.max_pages));
+      }
+      // A tile's rows take two dependent reads: its list entries, then the
+      // block-table entries they select.  Both are software-pipelined over
+      // the tiles: while tile pg's gathers go out, the block-table reads of
+      // tile pg + 2 and the list reads of tile pg + 3 are issued, and each
+      // value is first used one tile after its read was issued.  Lane l
+      // holds entries l and l + 32 of a tile.
+      auto load_pos = [&](int pg, int (&pos)[2]) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int e = pg * kPage + lane + 32 * k;
-          pos[k] = e < p.topk ? list[e] : -1;
+          pos[k] = (pg < p1 && e < p.topk) ? list[e] : -1;
         }
+      };
+      // -1 for a page outside the table (reported below if the entry is a key)
+      auto load_blk = [&](const int (&pos)[2], int (&blk)[2]) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int pgi = pos[k] / kPage;
+          blk[k] = (pos[k] >= 0 && pos[k] < L && pgi < p.max_pages) ? bt[pgi] : -1;
+        }
+      };
+      // cache rows (-1: not a key)
+      auto rows_of = [&](const int (&pos)[2], const int (&blk)[2], int (&row)[2]) {
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           row[k] = -1;
           if (pos[k] >= 0 && pos[k] < L) {
-            const int pgi = pos[k] / kPage;
-            const long long blk = pgi < p.max_pages ? bt[pgi] : -1;
-            if (blk < 0 || blk >= p.num_blocks) report_status(p.status, kStatusBadBlock);
-            else row[k] = static_cast<int>(blk) * kPage + pos[k] % kPage;
+            if (blk[k] < 0 || blk[k] >= p.num_blocks) report_status(p.status, kStatusBadBlock);
+            else row[k] = blk[k] * kPage + pos[k] % kPage;
           }
         }
       };
-      int cur[2], nxt[2] = {-1, -1};
-      if (p1 > p0) resolve(p0, cur);
+      int cur[2] = {-1, -1};
+      int pos1[2] = {-1, -1}, blk1[2] = {-1, -1}, pos2[2] = {-1, -1};  // tiles pg + 1 and pg + 2
+      if (p1 > p0) {
+        int pos0[2], blk0[2];
+        load_pos(p0, pos0);
+        load_pos(p0 + 1, pos1);
+        load_pos(p0 + 2, pos2);
+        load_blk(pos0, blk0);
+        load_blk(pos1, blk1);
+        rows_of(pos0, blk0, cur);
+      }
       for (int pg = p0; pg < p1; ++pg, ++g) {
-        const uint32_t st = g % kRawStages;
+        const uint32_t st = g % C::kRawStages;
         if (lane == 0) TRACE(kTraceProducer, g, 0);
-        if (pg + 1 < p1) resolve(pg + 1, nxt);  // its loads overlap the wait below
         int waited = 1;
-        if (lane == 0 && g >= static_cast<uint32_t>(kRawStages))
-          waited = mbar_wait(BAR(C::kRawEmpty + st), ((g / kRawStages) & 1u) ^ 1u, abort_flag, p.timeout_ns);
+        if (lane == 0 && g >= static_cast<uint32_t>(C::kRawStages))
+          waited = mbar_wait(BAR(C::kRawEmpty + st), ((g / C::kRawStages) & 1u) ^ 1u, abort_flag, p.timeout_ns);
         waited = __shfl_sync(0xffffffffu, waited, 0);
         if (!waited) {
           if (lane == 0) raise_abort(p, abort_flag);
@@ -453,27 +503,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           const int rr = t < 32 ? r0 : r1;
           rows[i] = rr < 0 ? 0 : rr;
         }
-        const uint32_t dst = rawbuf0 + st * kRawStageBytes;
+        const uint32_t dst = rawbuf0 + st * C::kRawStageBytes;
         if (lane < 16)
           tma_gather4(dst + q4 * 4 * 256, &tm_a, fb, static_cast<int>(rank) * 256, rows[0], rows[1], rows[2], rows[3]);
         else
           tma_gather4(dst + kRawLatBytes + q4 * 4 * kTailBytes, &tm_b, fb, kTailX, rows[0], rows[1], rows[2],
                       rows[3]);
-        cur[0] = nxt[0];
-        cur[1] = nxt[1];
         if (lane == 0) TRACE(kTraceProducer, g, 1);
+        // tile pg + 1's rows from reads issued a tile ago; the reads of the
+        // next two tiles go out
+        rows_of(pos1, blk1, cur);
+        load_blk(pos2, blk1);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) pos1[k] = pos2[k];
+        load_pos(pg + 3, pos2);
       }
     }
     // Never leave a copy landing in shared memory after the CTA exits.
     if (lane == 0)
-      for (uint32_t k = (g > static_cast<uint32_t>(kRawStages) ? g - kRawStages : 0u); k < g; ++k)
-        mbar_wait(BAR(C::kRawFull + k % kRawStages), (k / kRawStages) & 1u, &g_never_abort, 100000000ull);
+      for (uint32_t k = (g > static_cast<uint32_t>(C::kRawStages) ? g - C::kRawStages : 0u); k < g; ++k)
+        mbar_wait(BAR(C::kRawFull + k % C::kRawStages), (k / C::kRawStages) & 1u, &g_never_abort, 100000000ull);
   } else if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // BF16: page halves straight into the MMA stages.  FP8: raw bytes into
       // the raw stages, for the dequant warps.
-      constexpr int nst = kFp8 ? kRawStages : kStages;
+      constexpr int nst = kFp8 ? C::kRawStages : kStages;
       const int full0 = kFp8 ? C::kRawFull : C::kFull;
       const int empty0 = kFp8 ? C::kRawEmpty : C::kEmpty;
       uint32_t g = 0;
@@ -539,7 +594,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
           const int y = static_cast<int>(phys) * kPage;
           const uint32_t fb = BAR(full0 + st);
           if constexpr (kFp8) {
-            const uint32_t dst = rawbuf0 + st * kRawStageBytes;
+            const uint32_t dst = rawbuf0 + st * C::kRawStageBytes;
             mbar_arrive_expect_tx(fb, kRawBytes);
             tma_load_2d(dst, &tm_a, fb, static_cast<int>(rank) * 256, y);
             tma_load_2d(dst + kRawLatBytes, &tm_b, fb, 512, y);
@@ -1045,9 +1100,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
       const int L = p.seqlens[items[4 * it] / p.row_tiles / p.req_div];
       const int last_page = (L - 1) / kPage;
       for (int pg = p0; pg < p1; ++pg, ++g) {
-        const uint32_t rs = g % kRawStages, st = g % kStages;
+        const uint32_t rs = g % C::kRawStages, st = g % kStages;
         if (dt == 0) TRACE(kTraceDequant, g, 0);
-        if (!warp_wait(BAR(C::kRawFull + rs), (g / kRawStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!warp_wait(BAR(C::kRawFull + rs), (g / C::kRawStages) & 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
         if (dt == 0) TRACE(kTraceDequant, g, 1);
         if (g >= static_cast<uint32_t>(kStages) &&
             !warp_wait(BAR(C::kEmpty + st), ((g / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -1057,7 +1112,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
         const int valid = (pg == last_page) ? L - pg * kPage : kPage;
         uint64_t tmask = 0;
         if constexpr (kSparse) tmask = *reinterpret_cast<const volatile uint64_t*>(sbase + C::kRawMaskOffset + 8 * rs);
-        const uint8_t* rlat = sbase + C::kRawOffset + rs * kRawStageBytes;
+        const uint8_t* rlat = sbase + C::kRawOffset + rs * C::kRawStageBytes;
         // where token t's scales and this CTA's RoPE half are: the dense copy
         // lays them out as [64][16] and [64][64]; the sparse gather brings
         // bytes 496-655 of each token as one 160-byte row
@@ -1146,7 +1201,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
 template <bool kFp8, bool kSparse>
 static cudaError_t launch_decode(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_c,
                                  const DecodeParams& p, int num_parts, cudaStream_t stream) {
-  using C = dk::Cfg<kFp8>;
+  using C = dk::Cfg<kFp8, kSparse>;
   // The shared-memory opt-in is an attribute of the function on each device:
   // set it once per device (a bit per device below 64; devices above that set
   // it on every launch).  Racing host threads may both set it, which is

@@ -13,9 +13,12 @@
 // A split may therefore hold zero pages; the decode kernel then only writes
 // lse = -inf for it and the combine kernel gives it no weight.
 //
-// Whole-request mode: when batch <= parts and the costliest request is at
-// most kSplitPenaltyPages above t, part b serves request b alone (parts past
-// the batch stay idle) and nothing is split.
+// Whole-request mode: part k serves the m = ceil(batch / parts) requests
+// [k m, k m + m) whole (parts past the batch stay idle) and nothing is split,
+// when the costliest part is at most kSplitPenaltyPages above t.  (m = 1
+// when the batch fits the parts; m > 1 pays off for many equal requests,
+// such as the sparse decode's lists, where the balanced cut would split
+// nearly every request.)
 //
 // Requests with more than 128 query rows: everything above is over virtual
 // requests v = b * row_tiles + tile, each with the length of request b, so
@@ -103,11 +106,14 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
   __syncthreads();
   int t = max(1, (T + parts - 1) / parts);
 
-  // whole-request mode?
+  // whole-request mode?  The costliest part when part k takes requests
+  // [k m, k m + m) whole.
+  const int m = (batch + parts - 1) / parts;
   int local_max = 0;
-  for (int b = b0; b < b1; ++b) local_max = max(local_max, C[b + 1] - C[b]);
+  for (int k = threadIdx.x; k < parts; k += blockDim.x)
+    local_max = max(local_max, C[min((k + 1) * m, batch)] - C[min(k * m, batch)]);
   const int max_cost = block_max(local_max, warp_sums);
-  if (batch <= parts && max_cost <= t + kSplitPenaltyPages) {
+  if (max_cost <= t + kSplitPenaltyPages) {
     int32_t* part_first = sched + kSchedHeader;
     int32_t* items = sched + sched_items_offset(parts);
     for (int b = b0; b < b1; ++b) {
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__(kMetaThreads) metadata_kernel(const int32_t* _
       items[4 * b + 3] = -1;
       num_splits[b] = b;
     }
-    for (int k = threadIdx.x; k <= parts; k += blockDim.x) part_first[k] = min(k, batch);
+    for (int k = threadIdx.x; k <= parts; k += blockDim.x) part_first[k] = min(k * m, batch);
     if (threadIdx.x == 0) {
       num_splits[batch] = batch;
       sched[0] = parts;

@@ -26,8 +26,8 @@ import numpy as np
 PAGE = 64
 HEADER = 8
 DEFAULT_OVERHEAD = 4
-# Whole-request mode (one request per part, nothing split) is taken when the
-# batch fits the parts and the costliest request exceeds the balanced cut by
+# Whole-request mode (ceil(batch / parts) consecutive requests per part,
+# nothing split) is taken when the costliest part exceeds the balanced cut by
 # at most this many pages: splitting costs a round trip of fp32 partials, the
 # combine pass and a pipeline drain per extra item.
 SPLIT_PENALTY = 16
@@ -59,10 +59,13 @@ def plan(seqlens, parts: int, overhead: int = DEFAULT_OVERHEAD, rtiles: int = 1)
     C = np.concatenate([[0], np.cumsum(cost)])
     T = int(C[-1])
     t = max(1, -(-T // parts))
-    if B <= parts and int(cost.max(initial=0)) <= t + SPLIT_PENALTY:
+    m = max(1, -(-B // parts))  # requests per part in whole-request mode
+    firsts = np.minimum(np.arange(parts + 1) * m, B)
+    span = int((C[firsts[1:]] - C[firsts[:-1]]).max(initial=0))
+    if span <= t + SPLIT_PENALTY:
         sched = np.zeros(sched_ints(B, parts), dtype=np.int32)
-        sched[:8] = (parts, B, int(cost.max(initial=0)), B, overhead, 0, 1, rtiles)
-        sched[HEADER:HEADER + parts + 1] = np.minimum(np.arange(parts + 1), B)
+        sched[:8] = (parts, B, span, B, overhead, 0, 1, rtiles)
+        sched[HEADER:HEADER + parts + 1] = firsts
         io = items_offset(parts)
         items = np.stack([np.arange(B), np.zeros(B, dtype=np.int64), n, np.full(B, -1)], axis=1)
         sched[io:io + 4 * B] = items.reshape(-1)

@@ -62,6 +62,19 @@ def test_whole_requests_when_the_batch_fits():
     assert all(parts[b][0] == (b, 0, 64, -1) for b in range(64))
 
 
+def test_equal_requests_above_the_parts_stay_whole():
+    # 128 equal requests of 32 pages (the sparse decode's 2048-entry lists) on
+    # 74 CTA pairs: two whole requests per pair (72 units against a balanced
+    # cut of 63) instead of splitting nearly every request
+    L = [2048] * 128
+    sched, ns = schedule.plan(L, 74)
+    schedule.validate(sched, ns, L, 74)
+    assert int(sched[6]) == 1 and int(sched[5]) == 0 and int(sched[2]) == 72
+    parts = schedule.parse(sched, 74)
+    assert [len(x) for x in parts] == [2] * 64 + [0] * 10
+    assert all(parts[k] == [(2 * k, 0, 32, -1), (2 * k + 1, 0, 32, -1)] for k in range(64))
+
+
 def test_imbalanced_batch_is_still_split():
     # one request far above the balanced cut: splitting wins over the penalty
     L = [4096] * 63 + [65536]
