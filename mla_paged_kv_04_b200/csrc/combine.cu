@@ -16,25 +16,11 @@ namespace mla {
 constexpr int kCombineWarps = 4;  // one query row per warp
 constexpr int kCombineUnroll = 4;  // splits whose partial rows are in flight at once
 
-// grid.x walks the schedule's list of split (virtual) requests (at most one per CTA
-// pair), grid.y covers the query rows four at a time, one row per warp.  Lane
-// s holds split s's weight (in chunks of 32 splits); the partial rows of
-// kCombineUnroll splits are loaded together so that their latencies overlap.
-__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineParams p) {
-  pdl_wait();  // the decode kernel has completed
-  // a schedule made for another CTA-pair count or batch: reported by the
-  // decode kernel, nothing to merge
-  if (p.sched[0] != p.num_parts || p.sched[3] != p.batch * p.row_tiles || p.sched[7] != p.row_tiles) return;
-  const int num_split_req = p.sched[5];
-  if (static_cast<int>(blockIdx.x) >= num_split_req) return;
-  const int parts = p.sched[0];
-  const int vb = p.sched[sched_split_list_offset(parts) + blockIdx.x];  // virtual request
+// Merges row r of split virtual request vb (one warp).
+__device__ __forceinline__ void combine_row(const CombineParams& p, int vb, int r, int mt, int lane) {
   const int b = vb / p.row_tiles, row0 = (vb - b * p.row_tiles) * kRows;
-  const int mt = rows_per_tile(p.M);  // partial rows per slot
   const int first = p.num_splits[vb];
   const int nsplit = p.num_splits[vb + 1] - first;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y * kCombineWarps + warp;  // row within the row tile
   if (r >= mt || row0 + r >= p.M) return;
 
   float m = -CUDART_INF_F;
@@ -98,9 +84,37 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const Combi
   if (lane == 0) p.lse[orow] = wsum > 0.f ? m + logf(wsum) : -CUDART_INF_F;
 }
 
+// At most this many blocks: when no request is split (whole-request
+// schedules) the kernel's cost is its launch and drain, which grows with the
+// grid; otherwise blocks loop over the work.
+constexpr int kCombineMaxBlocks = 4 * 148;
+
+// One work unit per (split virtual request, group of kCombineWarps query
+// rows), one row per warp; blocks take units blockIdx.x, blockIdx.x +
+// gridDim.x, ...  Lane s holds split s's weight (in chunks of 32 splits); the
+// partial rows of kCombineUnroll splits are loaded together so that their
+// latencies overlap.
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const CombineParams p) {
+  pdl_wait();  // the decode kernel has completed
+  // a schedule made for another CTA-pair count or batch: reported by the
+  // decode kernel, nothing to merge
+  if (p.sched[0] != p.num_parts || p.sched[3] != p.batch * p.row_tiles || p.sched[7] != p.row_tiles) return;
+  const int num_split_req = p.sched[5];
+  const int parts = p.sched[0];
+  const int mt = rows_per_tile(p.M);  // partial rows per slot
+  const int groups = (mt + kCombineWarps - 1) / kCombineWarps;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int unit = blockIdx.x; unit < num_split_req * groups; unit += gridDim.x) {
+    const int vb = p.sched[sched_split_list_offset(parts) + unit / groups];  // virtual request
+    const int r = (unit % groups) * kCombineWarps + warp;                     // row within the row tile
+    combine_row(p, vb, r, mt, lane);
+  }
+}
+
 cudaError_t launch_combine(const CombineParams& p, int parts, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(parts, (rows_per_tile(p.M) + kCombineWarps - 1) / kCombineWarps);
+  const int units = parts * ((rows_per_tile(p.M) + kCombineWarps - 1) / kCombineWarps);  // upper bound
+  cfg.gridDim = dim3(units < kCombineMaxBlocks ? units : kCombineMaxBlocks);
   cfg.blockDim = dim3(32 * kCombineWarps);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
