@@ -358,7 +358,6 @@ mla_status_t mla_sparse_decode_fwd(const void* q, const void* kv_cache, int64_t 
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
   p.req_div = s_q;
   p.req_batch = batch;
-  p.kv_raw = static_cast<const uint8_t*>(kv_cache);
   p.indices = indices;
   p.topk = topk;
   p.q_wide = aligned(q, 32) ? 1 : 0;

@@ -111,7 +111,6 @@ struct DecodeParams {
   // and the block table and the lengths are indexed by unit / req_div.
   int req_div;
   int req_batch;                // rows of block_table and seqlens
-  const uint8_t* kv_raw;        // sparse: the 656-byte cache, read with bulk copies
   const int32_t* indices;       // sparse: [batch units, topk] positions in the request
   int topk;
 };
