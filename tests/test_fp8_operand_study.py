@@ -1,0 +1,78 @@
+"""Accuracy study for an FP8-operand QK^T (tensor-core kind::f8f6f4), on the CPU.
+
+A QK^T on FP8 operands would need q in E4M3 as well as the cache's codes.  The
+CUTLASS discussion page ("Unified E4M3 format", activations grouped and
+scaled on 1x128 tiles) describes the usual scheme: each 128-wide group of a
+row gets an fp32 scale amax / 448 and its values are rounded to E4M3.  This
+study applies that to q (the latent dims in four groups of 128, the 64 RoPE
+dims as a fifth group) and keeps every other step exact, so the errors
+measured are a lower bound for any FP8-operand kernel.  References are the
+float64 oracle on the exact keys.
+
+Finding (asserted below, request lengths 16 / 256 / 8192): E4M3 keeps 3
+mantissa bits, so each q element moves by up to 2^-4 of itself and the
+logits by a few hundredths (softmax units) on N(0,1) data.  The lse error is
+0.025 / 0.010 / 0.0054: 5 to 25 times the 1e-3 tolerance at every length (a
+softmax leans on its largest logits, so long rows do not average the error
+away), and the output error on the 16-key row (0.057) is also above its 2e-2
+bound.  The bf16 pipeline (q exact, keys rounded once to bf16) stays inside
+the tolerance from 256 keys on (0.00057 / 0.00009); on 16 keys its rounding
+alone reaches 0.0014, which is why the FP8 parity tests feed the oracle the
+kernel's own dequantised cache (reading R8).  The FP8-operand variant is not
+built: its q rounding alone breaks the lse tolerance on every row length.
+"""
+
+import numpy as np
+import torch
+
+import oracle
+from oracle import mla as om
+import workloads as W
+
+LSE_TOL = 1e-3
+
+
+def _quantize_groups_e4m3(x: np.ndarray, bounds) -> np.ndarray:
+    """Per-group E4M3 rounding of the last axis: scale = amax / 448 (fp32),
+    value = e4m3(x / scale) * scale.  An all-zero group stays zero."""
+    out = np.empty_like(x)
+    for lo, hi in bounds:
+        g = x[..., lo:hi]
+        amax = np.abs(g).max(axis=-1, keepdims=True)
+        scale = (amax / 448.0).astype(np.float32).astype(np.float64)
+        safe = np.where(scale > 0, scale, 1.0)
+        codes = om.encode_e4m3_rne((g / safe).astype(np.float32))
+        out[..., lo:hi] = np.where(scale > 0, om.decode_e4m3(codes) * safe, 0.0)
+    return out
+
+
+def _max_errs(q, keys, L, scale, ref_out, ref_lse):
+    out, lse = oracle.mla_decode_partial(q, keys, L, scale, False, 0, L)
+    return float(np.abs(lse - ref_lse).max()), float(np.abs(out - ref_out).max())
+
+
+def test_e4m3_q_breaks_the_lse_tolerance():
+    w = W.Workload("study", 3, 1, 128, (1, 1), fmt="fp8_656", seed=51)
+    lengths = [16, 256, 8192]
+    c = W.make_case(w, seqlens=lengths, poison=False)
+    a = W.oracle_arrays(c)
+    groups = [(0, 128), (128, 256), (256, 384), (384, 512), (512, 576)]
+    errs_fp8, outs_fp8, errs_bf16 = [], [], []
+    for b, L in enumerate(lengths):
+        q = oracle.decode_bf16_bits(a["q_bits"][b])  # [1, 128, 576]
+        keys = oracle.gather_keys(a["kv_cache"], "fp8_656", a["block_table"][b], L)
+        ref_out, ref_lse = oracle.mla_decode_partial(q, keys, L, a["softmax_scale"], False, 0, L)
+        q8 = _quantize_groups_e4m3(q, groups)
+        e, o = _max_errs(q8, keys, L, a["softmax_scale"], ref_out, ref_lse)
+        errs_fp8.append(e)
+        outs_fp8.append(o)
+        # the bf16 pipeline: exact q, keys rounded once to bf16
+        kb = torch.from_numpy(keys).to(torch.bfloat16).double().numpy()
+        errs_bf16.append(_max_errs(q, kb, L, a["softmax_scale"], ref_out, ref_lse)[0])
+    # E4M3 q: outside the lse tolerance at every length, and the 16-key row's
+    # output outside its bound too
+    assert all(e > 5 * LSE_TOL for e in errs_fp8), errs_fp8
+    assert outs_fp8[0] > 2e-2, outs_fp8
+    # bf16 keys: inside the tolerance once rows hold a few hundred keys
+    assert all(e <= LSE_TOL for e in errs_bf16[1:]), errs_bf16
+    assert all(e < f / 10 for e, f in zip(errs_bf16, errs_fp8)), (errs_bf16, errs_fp8)
