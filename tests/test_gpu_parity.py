@@ -186,6 +186,54 @@ def test_metadata_covers_every_page_once():
         np.testing.assert_array_equal(dev_sched[io:used], host_sched[io:used])
 
 
+def _same_schedule(dev_sched, dev_ns, host_sched, host_ns, parts):
+    np.testing.assert_array_equal(dev_ns, host_ns)
+    np.testing.assert_array_equal(dev_sched[:8 + parts + 1], host_sched[:8 + parts + 1])
+    off, nsr = schedule_mod().split_list_offset(parts), int(host_sched[5])
+    np.testing.assert_array_equal(dev_sched[off:off + nsr], host_sched[off:off + nsr])
+    io = schedule_mod().items_offset(parts)
+    used = io + 4 * int(host_sched[1])
+    np.testing.assert_array_equal(dev_sched[io:used], host_sched[io:used])
+
+
+def schedule_mod():
+    from mla_paged_kv_04_b200 import schedule
+    return schedule
+
+
+@pytest.mark.parametrize("lengths,parts", [([2048] * 128, 74), ([640] * 300, 74), ([100, 90, 80, 70, 60], 2)])
+def test_metadata_whole_requests_several_per_pair(lengths, parts):
+    """Equal requests above the CTA-pair count: the device schedule takes the
+    whole-request mode with ceil(batch / parts) requests per pair, exactly as
+    the host planner does."""
+    import mla_paged_kv_04_b200 as mla
+    schedule = schedule_mod()
+    L = torch.tensor(lengths, dtype=torch.int32)
+    sched, ns = mla.mla_get_metadata(L.cuda(), 1, 128, parts)
+    torch.cuda.synchronize()
+    dev_sched, dev_ns = sched.cpu().numpy(), ns.cpu().numpy()
+    schedule.validate(dev_sched, dev_ns, L.numpy(), parts)
+    host_sched, host_ns = schedule.plan(L.numpy(), parts)
+    assert int(host_sched[6]) == 1
+    _same_schedule(dev_sched, dev_ns, host_sched, host_ns, parts)
+
+
+@pytest.mark.parametrize("batch,s_q,h_q,topk,parts", [(128, 1, 128, 2048, 74), (3, 2, 200, 300, 5), (40, 4, 64, 64, 74)])
+def test_sparse_metadata_matches_the_host_planner(batch, s_q, h_q, topk, parts):
+    """The sparse schedule plans batch * s_q units of h_q rows (row tiles of
+    128), each of length topk, like the dense planner with equal lengths."""
+    import mla_paged_kv_04_b200 as mla
+    schedule = schedule_mod()
+    sched, ns = mla.mla_get_sparse_metadata(batch, s_q, h_q, topk, parts, device="cuda")
+    torch.cuda.synchronize()
+    rt = schedule.row_tiles(1, h_q)
+    lengths = np.full(batch * s_q, topk)
+    dev_sched, dev_ns = sched.cpu().numpy(), ns.cpu().numpy()
+    schedule.validate(dev_sched, dev_ns, lengths, parts, rtiles=rt)
+    host_sched, host_ns = schedule.plan(lengths, parts, rtiles=rt)
+    _same_schedule(dev_sched, dev_ns, host_sched, host_ns, parts)
+
+
 @pytest.mark.parametrize("name", W.ORDER)
 def test_full_size_every_request(name):
     """Each configured workload at full size, in the launch configuration the
