@@ -1,11 +1,11 @@
 /*
  * mla.h — C ABI of the B200 (sm_100a) MLA paged-KV decoding library.
  *
- * Operation (FlashMLA, described on the pages as an "efficient MLA decoding
- * kernel ... optimized for variable-length sequences", BF16, "Paged KV cache
- * (block size 64)": DeepSeek launch tweet quoted on the 8bitnewsroom page;
- * MLA's shared compressed latent KV with decoupled RoPE: Novita AI page,
- * section "Was ist MLA?" and its MHA/MQA/GQA/MLA table):
+ * Operation (FlashMLA, an MLA decoding kernel for batches of
+ * variable-length sequences over a BF16 cache paged in 64-token blocks, as
+ * the DeepSeek launch tweet on the 8bitnewsroom page describes it; MLA's
+ * shared compressed latent KV with decoupled RoPE: Novita AI page, section
+ * "Was ist MLA?" and its MHA/MQA/GQA/MLA table):
  *
  *   For request b with L = cache_seqlens[b] cached tokens, query token i in
  *   [0, s_q) and head h in [0, h_q):
@@ -85,9 +85,9 @@ size_t mla_metadata_size(int batch, int s_q, int h_q, int num_sm_parts);
 int mla_num_splits_len(int batch, int s_q, int h_q);
 
 /*
- * Split-KV schedule (the split-KV idea follows from "optimized for
- * variable-length sequences" on the 8bitnewsroom page; the pages give no
- * algorithm, this one is our own).  Every request costs ceil(L/64) pages
+ * Split-KV schedule (the split-KV idea follows from the variable-length
+ * batches the 8bitnewsroom page names as FlashMLA's target; the pages give
+ * no algorithm, this one is our own).  Every request costs ceil(L/64) pages
  * plus a fixed per-request overhead; the concatenated cost line is cut into
  * num_sm_parts equal pieces, so a request may be split across CTA pairs.
  * When batch <= num_sm_parts and the costliest request exceeds the balanced

@@ -8,9 +8,9 @@ the only thing both sides see is the seeded input generator in ``workloads``,
 which holds none of the method's arithmetic.
 
 Every function is a plain restatement of what the method computes, written
-from the descriptions of FlashMLA ("efficient MLA decoding kernel for Hopper
-GPUs ... BF16 ... paged KV cache (block size 64)", DeepSeek launch tweet on
-the 8bitnewsroom page; MLA's shared latent KV with decoupled RoPE, Novita AI
+from the descriptions of FlashMLA (an MLA decoding kernel for Hopper GPUs
+over a BF16 cache paged in 64-token blocks, DeepSeek launch tweet on the
+8bitnewsroom page; MLA's shared latent KV with decoupled RoPE, Novita AI
 page, section "Was ist MLA?" and its MHA/MQA/GQA/MLA table; the 656-byte FP8
 cache format, menfem.com DeepSeek page, "Key Contributions").  Where those
 pages are silent the reading taken is stated in the docstring.

@@ -9,9 +9,8 @@ What is computed (MLA decode, FlashMLA pages):
     table).  Each cached token is a 576-wide key: a 512-d latent followed by a
     64-d decoupled-RoPE slice.  The value of a token is the first 512 dims of
     its key (the latent).
-  * The cache is paged with 64 tokens per block (DeepSeek launch tweet,
-    8bitnewsroom page: "Paged KV cache (block size 64)") and requests have
-    variable lengths ("optimized for variable-length sequences", same tweet).
+  * The cache is paged with 64 tokens per block and requests have variable
+    lengths (DeepSeek launch tweet, 8bitnewsroom page).
   * Two cache formats: BF16 (576 x 2 = 1152 bytes per token) and FP8 at 656
     bytes per token with the RoPE slice kept in BF16 (menfem.com DeepSeek
     page, "Key Contributions").

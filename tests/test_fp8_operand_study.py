@@ -1,8 +1,8 @@
 """Accuracy study for an FP8-operand QK^T (tensor-core kind::f8f6f4), on the CPU.
 
 A QK^T on FP8 operands would need q in E4M3 as well as the cache's codes.  The
-CUTLASS discussion page ("Unified E4M3 format", activations grouped and
-scaled on 1x128 tiles) describes the usual scheme: each 128-wide group of a
+CUTLASS discussion page describes the usual scheme, one E4M3 format for all
+operands with activations scaled per 1x128 tile: each 128-wide group of a
 row gets an fp32 scale amax / 448 and its values are rounded to E4M3.  This
 study applies that to q (the latent dims in four groups of 128, the 64 RoPE
 dims as a fifth group) and keeps every other step exact, so the errors

@@ -6,8 +6,8 @@ numbers, lays them out in the cache formats and builds page tables.
 
 The five workloads follow the configured benchmark set (tiny; uniform BF16;
 variable-length speculative BF16; FP8 656-byte cache; long context).  The
-pages describe no dataset, only "variable-length sequences", a paged cache
-with 64-token blocks (DeepSeek launch tweet, 8bitnewsroom page) and a Novita
+pages describe no dataset, only batches of variable-length sequences over a
+cache paged in 64-token blocks (DeepSeek launch tweet, 8bitnewsroom page) and a Novita
 AI sweep over batch size, sequence length and head count whose charts did not
 survive; these generators stand in for all of them.
 
