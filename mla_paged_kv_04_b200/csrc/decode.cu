@@ -24,6 +24,11 @@
 //     swizzled tile the QK^T product reads as K-major.
 //   * Epilogue: bf16 out + lse for an unsplit request, fp32 partials for a
 //     split one (merged by the combine kernel).
+//   * Sparse variant (FP8 cache): a unit is one query token, and its tiles are
+//     64-entry slices of its index list instead of pages.  The producer is a
+//     whole warp that maps the listed positions through the block table and
+//     gathers the rows with TMA; a per-tile validity mask replaces the length
+//     mask.
 //
 // Warp roles: warp 0 TMA producer, warp 1 QK^T issuer, warp 2 tensor-memory
 // allocator, warp 3 PV issuer; warps 4-11 softmax in two warpgroups that take
@@ -36,9 +41,9 @@
 // read without waiting (any reference is correct; the two converge within a
 // tile or two).  The combined reference of the last consumed tile, which is
 // the scale O is at, passes between them through an mbarrier-guarded slot, so
-// O is rescaled exactly when that scale moves.  tcgen05.mma issue blocks for about the
-// instruction's run time, so QK^T and PV get one issuing thread each (one
-// thread for both would hold QK^T(j + 1) behind PV(j)), with their
+// O is rescaled exactly when that scale moves.  tcgen05.mma issue blocks for
+// about the instruction's run time, so QK^T and PV get one issuing thread each
+// (one thread for both would hold QK^T(j + 1) behind PV(j)), with their
 // shared-memory descriptors precomputed.
 //
 // Every mbarrier wait is bounded (params.timeout_ns); a wait that runs out
@@ -392,7 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(dk::Cfg<kFp8>::kThre
     // list.  Lane l resolves entries l and l + 32: it reads the position,
     // checks it against the request's length and maps it through the block
     // table to a row of the cache (viewed as [num_blocks * 64, 656] bytes).
-    // These reads run one tile ahead of the copies.  The copies are TMA
+    // These reads run ahead of the copies (see below).  The copies are TMA
     // gathers of four rows: lanes 0-15 bring the latent halves of tokens
     // 4l .. 4l + 3 (256 bytes each), lanes 16-31 their tails (bytes 496-655).
     // Entries that are not keys (padding, positions outside [0, L), pages that

@@ -132,14 +132,6 @@ __device__ __forceinline__ void st_global_v8(void* p, uint32_t a, uint32_t b, ui
                ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d), "r"(e), "r"(f), "r"(g), "r"(h)
                : "memory");
 }
-// Non-tensor bulk copy global -> this CTA's shared memory, completing on an
-// mbarrier (16-byte aligned addresses, size a multiple of 16).
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
 // TMA gather of four rows of a 2-D tensor map whose box is one row high:
 // the boxes at (x, y0) .. (x, y3) land one after another at dst.  x times the
 // element size must be a multiple of 16 bytes.
