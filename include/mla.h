@@ -90,9 +90,10 @@ int mla_num_splits_len(int batch, int s_q, int h_q);
  * no algorithm, this one is our own).  Every request costs ceil(L/64) pages
  * plus a fixed per-request overhead; the concatenated cost line is cut into
  * num_sm_parts equal pieces, so a request may be split across CTA pairs.
- * When batch <= num_sm_parts and the costliest request exceeds the balanced
- * cut by at most 16 pages, every request gets a CTA pair of its own instead
- * and nothing is split (no partial outputs, no combine work).
+ * When giving each CTA pair ceil(batch / num_sm_parts) consecutive whole
+ * requests makes no pair's cost exceed the balanced cut by more than 16
+ * pages, that is done instead and nothing is split (no partial outputs, no
+ * combine work).
  *
  *   cache_seqlens  device int32 [batch], each >= 0
  *   s_q, h_q       query tokens and heads per request: they fix the row
@@ -180,9 +181,10 @@ mla_status_t mla_decode_fwd(const void* q, const void* kv_cache, mla_kv_format_t
  *                  topk, num_sm_parts): a schedule of batch * s_q units of
  *                  h_q rows, each of length topk
  *   out, lse       as mla_decode_fwd;  workspace >= mla_sparse_workspace_size()
- * Each CTA pair gathers the listed tokens of a 64-entry tile with bulk
- * copies (this CTA's 336 bytes of each token), dequantises them like the
- * dense FP8 decode and runs the same MMA and softmax pipeline.  Device-
+ * Each CTA pair gathers the listed tokens of a 64-entry tile with TMA row
+ * gathers (per CTA, its 256 latent bytes and bytes 496-655 of each token),
+ * dequantises them like the dense FP8 decode and runs the same MMA and
+ * softmax pipeline.  Device-
  * detected errors as mla_decode_fwd (a listed position whose page maps
  * outside [0, num_blocks): MLA_ERR_BAD_BLOCK_INDEX, that entry left out).
  */
